@@ -1,0 +1,270 @@
+/*
+ * nvfp4kv_oracle.cpp -- CPU oracle for the NVFP4 KV-cache path.
+ *
+ * TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the benchmark's CPU
+ * baseline load this file's library; the CUDA library never does.  It is deliberately
+ * plain and slow: one thread, scalar loops, no blocking or reordering beyond what the
+ * definitions state.  Build with -O2 -ffp-contract=off and without fast-math so that
+ * every fp32 operation below is one IEEE-754 round-to-nearest-even operation.
+ *
+ * What it computes (sources cited as in nvfp4kv_oracle.h):
+ *
+ *  NVFP4 quantisation of one K or V chunk of one head [P1 sec. 2.2], [N1], [N2]:
+ *   The pages lose the equation itself; only its constants (16-element blocks,
+ *   M_FP8 = 448, M_FP4 = 6) and the three factors of dequantisation survive.  The reading
+ *   taken here, in fp32 with round-to-nearest-even at every step:
+ *     A      = max |x| over the chunk (exact)
+ *     g      = A / (448 * 6)                       (0 when A == 0)      -- FP32 scale
+ *     for every token and every 16-element block b along the head dimension:
+ *       a_b  = max |x| over the block
+ *       s    = E4M3(a_b / (6 * g))                 (0 when a_b == 0 or g == 0) -- block scale
+ *       r    = 1 / (decode(s) * g)
+ *       q_i  = E2M1(x_i * r)                       (all 0 when decode(s) == 0 or r is not finite)
+ *   E4M3() and E2M1() round to the nearest representable value, ties to the even code,
+ *   and clamp to the largest finite magnitude.
+ *  Dequantisation [N1]: x_hat = E2M1(q) * E4M3(s) * g, evaluated in fp64 (exact).
+ *  Attention [P1' sec. 4.2], [P1'' sec. 2.1]: a query row of chunk t attends to the keys of
+ *   the visible chunks V(t) = {c < n_sink} U {t - window < c <= t} (duplicates removed), in
+ *   fp64: s_j = sigma * q . k_hat_j, p_j = exp(s_j - max_j s_j), o = sum p_j v_hat_j / sum p_j.
+ */
+#include "nvfp4kv_oracle.h"
+
+#include <cmath>
+#include <cstring>
+#include <limits>
+#include <vector>
+#include <xmmintrin.h>
+
+namespace {
+
+/* Keep subnormals: clear flush-to-zero and denormals-are-zero for the duration of a call. */
+struct IeeeMode {
+  unsigned saved;
+  IeeeMode() : saved(_mm_getcsr()) { _mm_setcsr(saved & ~(0x8000u | 0x0040u)); }
+  ~IeeeMode() { _mm_setcsr(saved); }
+};
+
+float bf16_bits_to_float(uint16_t h) {
+  uint32_t u = static_cast<uint32_t>(h) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+/* Nearest code among the ascending non-negative magnitudes dec(0) < dec(1) < ... <
+ * dec(n-1); an exact tie goes to the even code; anything at or beyond the largest
+ * magnitude takes the largest code. */
+uint8_t nearest_magnitude_code(double a, int n, double (*dec)(uint8_t)) {
+  const double top = dec(static_cast<uint8_t>(n - 1));
+  if (a >= top) return static_cast<uint8_t>(n - 1);
+  int best = 0;
+  double best_d = std::fabs(a - dec(0));
+  for (int c = 1; c < n; ++c) {
+    const double dist = std::fabs(a - dec(static_cast<uint8_t>(c)));
+    if (dist < best_d || (dist == best_d && (c % 2) == 0)) {
+      best = c;
+      best_d = dist;
+    }
+  }
+  return static_cast<uint8_t>(best);
+}
+
+double e2m1_magnitude(uint8_t c) { return oracle_e2m1_decode(static_cast<uint8_t>(c & 7)); }
+double e4m3_magnitude(uint8_t c) { return oracle_e4m3_decode(static_cast<uint8_t>(c & 0x7F)); }
+
+}  // namespace
+
+extern "C" {
+
+/* E2M1: bit 3 sign, bits 2..1 exponent (bias 1), bit 0 mantissa [N1 "The NVFP4
+ * quantization format"]; exponent 0 is the subnormal 0.5 * m. */
+double oracle_e2m1_decode(uint8_t code) {
+  const int e = (code >> 1) & 3;
+  const int m = code & 1;
+  const double mag = (e == 0) ? 0.5 * m : std::ldexp(1.0 + 0.5 * m, e - 1);
+  return (code & 8) ? -mag : mag;
+}
+
+uint8_t oracle_e2m1_encode(float v) {
+  const uint8_t sign = std::signbit(v) ? 8 : 0;
+  /* 8 magnitudes (codes 0..7), largest 6 = M_FP4 [P1 sec. 2.2]. */
+  return static_cast<uint8_t>(sign | nearest_magnitude_code(std::fabs(static_cast<double>(v)), 8,
+                                                            e2m1_magnitude));
+}
+
+/* E4M3: bit 7 sign, bits 6..3 exponent (bias 7), bits 2..0 mantissa; exponent 0 is
+ * subnormal (m * 2^-9); S.1111.111 is NaN, so the largest finite magnitude is
+ * 1.75 * 2^8 = 448 = M_FP8 [P1 sec. 2.2]. */
+double oracle_e4m3_decode(uint8_t code) {
+  const int e = (code >> 3) & 15;
+  const int m = code & 7;
+  if (e == 15 && m == 7) return std::numeric_limits<double>::quiet_NaN();
+  const double mag = (e == 0) ? std::ldexp(static_cast<double>(m), -9)
+                              : std::ldexp(1.0 + m / 8.0, e - 7);
+  return (code & 0x80) ? -mag : mag;
+}
+
+uint8_t oracle_e4m3_encode(float v) {
+  const uint8_t sign = std::signbit(v) ? 0x80 : 0;
+  /* 127 finite magnitudes, codes 0x00..0x7E. */
+  return static_cast<uint8_t>(sign | nearest_magnitude_code(std::fabs(static_cast<double>(v)), 127,
+                                                            e4m3_magnitude));
+}
+
+int oracle_quantize_chunk(const uint16_t* x, int32_t B, int32_t L, int32_t H, int32_t d,
+                          int64_t token_stride, uint8_t* codes, uint8_t* scales, float* gscale) {
+  if (!x || !codes || !scales || !gscale || B <= 0 || L <= 0 || H <= 0 || d <= 0 || d % 16 != 0 ||
+      token_stride < static_cast<int64_t>(H) * d)
+    return -1;
+  IeeeMode ieee;
+  const int nblk = d / 16;
+  const float kFp8Max = 448.0f;  /* M_FP8 */
+  const float kFp4Max = 6.0f;    /* M_FP4 */
+  for (int32_t b = 0; b < B; ++b) {
+    for (int32_t h = 0; h < H; ++h) {
+      auto elem = [&](int32_t t, int32_t i) {
+        return bf16_bits_to_float(x[(static_cast<int64_t>(b) * L + t) * token_stride +
+                                    static_cast<int64_t>(h) * d + i]);
+      };
+      /* FP32 scale of this (chunk, head). */
+      float A = 0.0f;
+      for (int32_t t = 0; t < L; ++t)
+        for (int32_t i = 0; i < d; ++i) A = std::fmax(A, std::fabs(elem(t, i)));
+      const float g = (A == 0.0f) ? 0.0f : A / (kFp8Max * kFp4Max);
+      gscale[static_cast<int64_t>(b) * H + h] = g;
+
+      const int64_t row0 = (static_cast<int64_t>(b) * H + h) * L;
+      for (int32_t t = 0; t < L; ++t) {
+        uint8_t* crow = codes + (row0 + t) * (d / 2);
+        uint8_t* srow = scales + (row0 + t) * nblk;
+        std::memset(crow, 0, static_cast<size_t>(d / 2));
+        for (int blk = 0; blk < nblk; ++blk) {
+          float ab = 0.0f;
+          for (int k = 0; k < 16; ++k) ab = std::fmax(ab, std::fabs(elem(t, blk * 16 + k)));
+          uint8_t s_code = 0;
+          if (ab != 0.0f && g != 0.0f) {
+            const float denom = kFp4Max * g;
+            const float s_raw = ab / denom;
+            s_code = oracle_e4m3_encode(s_raw);
+          }
+          srow[blk] = s_code;
+          const float s = static_cast<float>(oracle_e4m3_decode(s_code));
+          if (s == 0.0f) continue; /* codes stay 0 */
+          const float sg = s * g;
+          const float r = 1.0f / sg;
+          if (!std::isfinite(r)) continue; /* scale product underflowed: codes stay 0 */
+          for (int k = 0; k < 16; ++k) {
+            const int i = blk * 16 + k;
+            const float y = elem(t, i) * r;
+            const uint8_t q = oracle_e2m1_encode(y);
+            crow[i / 2] |= static_cast<uint8_t>((i % 2 == 0) ? q : (q << 4));
+          }
+        }
+      }
+    }
+  }
+  return 0;
+}
+
+int oracle_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gscale, int32_t B,
+                      int32_t H, int32_t d, int32_t chunk_tokens, int32_t capacity, double* out) {
+  if (!codes || !scales || !gscale || !out || B <= 0 || H <= 0 || d <= 0 || d % 16 != 0 ||
+      chunk_tokens <= 0 || capacity <= 0)
+    return -1;
+  const int64_t T = static_cast<int64_t>(chunk_tokens) * capacity;
+  for (int32_t b = 0; b < B; ++b)
+    for (int32_t h = 0; h < H; ++h)
+      for (int64_t t = 0; t < T; ++t) {
+        const int64_t row = (static_cast<int64_t>(b) * H + h) * T + t;
+        const double g = gscale[(static_cast<int64_t>(b) * H + h) * capacity + t / chunk_tokens];
+        for (int32_t i = 0; i < d; ++i) {
+          const uint8_t byte = codes[row * (d / 2) + i / 2];
+          const uint8_t q = (i % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+          const double s = oracle_e4m3_decode(scales[row * (d / 16) + i / 16]);
+          out[row * d + i] = oracle_e2m1_decode(q) * s * g;
+        }
+      }
+  return 0;
+}
+
+int oracle_visible_chunks(int32_t q_chunk, int32_t n_sink, int32_t window, int32_t capacity,
+                          int32_t* out) {
+  if (!out || capacity <= 0 || q_chunk < 0 || q_chunk >= capacity || n_sink < 0 || window < 1)
+    return -1;
+  int n = 0;
+  for (int32_t c = 0; c < capacity; ++c) {
+    const bool in_sink = c < n_sink;                             /* A_g */
+    const bool in_window = (c > q_chunk - window) && (c <= q_chunk); /* sliding window */
+    if (in_sink || in_window) out[n++] = c;                      /* union: each chunk once */
+  }
+  return n;
+}
+
+int oracle_attention_rows(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, int32_t d,
+                          int64_t q_token_stride,
+                          const uint8_t* k_codes, const uint8_t* k_scales, const float* k_gscale,
+                          const uint8_t* v_codes, const uint8_t* v_scales, const float* v_gscale,
+                          int32_t chunk_tokens, int32_t capacity,
+                          int32_t q_chunk, int32_t n_sink, int32_t window, double softmax_scale,
+                          const int32_t* rows, int32_t n_rows, double* out) {
+  if (!q || !k_codes || !k_scales || !k_gscale || !v_codes || !v_scales || !v_gscale || !rows ||
+      !out || B <= 0 || Lq <= 0 || H <= 0 || d <= 0 || d % 16 != 0 || chunk_tokens <= 0 ||
+      capacity <= 0 || n_rows < 0 || q_token_stride < static_cast<int64_t>(H) * d)
+    return -1;
+  std::vector<int32_t> vis(static_cast<size_t>(capacity));
+  const int nvis = oracle_visible_chunks(q_chunk, n_sink, window, capacity, vis.data());
+  if (nvis < 0) return -1;
+  const double sigma = softmax_scale > 0.0 ? softmax_scale : 1.0 / std::sqrt(static_cast<double>(d));
+  const int64_t T = static_cast<int64_t>(chunk_tokens) * capacity;
+
+  /* x_hat of one cached token (fp64, exact). */
+  auto dequant_row = [&](const uint8_t* codes, const uint8_t* scales, const float* gs, int32_t b,
+                         int32_t h, int64_t t, double* dst) {
+    const int64_t row = (static_cast<int64_t>(b) * H + h) * T + t;
+    const double g = gs[(static_cast<int64_t>(b) * H + h) * capacity + t / chunk_tokens];
+    for (int32_t i = 0; i < d; ++i) {
+      const uint8_t byte = codes[row * (d / 2) + i / 2];
+      const uint8_t c = (i % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+      dst[i] = oracle_e2m1_decode(c) * oracle_e4m3_decode(scales[row * (d / 16) + i / 16]) * g;
+    }
+  };
+
+  std::vector<double> qrow(static_cast<size_t>(d)), krow(static_cast<size_t>(d)),
+      vrow(static_cast<size_t>(d)), o(static_cast<size_t>(d));
+  std::vector<double> s;
+  for (int32_t r = 0; r < n_rows; ++r) {
+    const int32_t b = rows[3 * r + 0], h = rows[3 * r + 1], i = rows[3 * r + 2];
+    if (b < 0 || b >= B || h < 0 || h >= H || i < 0 || i >= Lq) return -1;
+    for (int32_t e = 0; e < d; ++e)
+      qrow[e] = bf16_bits_to_float(q[(static_cast<int64_t>(b) * Lq + i) * q_token_stride +
+                                     static_cast<int64_t>(h) * d + e]);
+    /* pass 1: logits over every visible key */
+    s.clear();
+    for (int n = 0; n < nvis; ++n)
+      for (int32_t j = 0; j < chunk_tokens; ++j) {
+        const int64_t t = static_cast<int64_t>(vis[n]) * chunk_tokens + j;
+        dequant_row(k_codes, k_scales, k_gscale, b, h, t, krow.data());
+        double dot = 0.0;
+        for (int32_t e = 0; e < d; ++e) dot += qrow[e] * krow[e];
+        s.push_back(sigma * dot);
+      }
+    double smax = -std::numeric_limits<double>::infinity();
+    for (double v : s) smax = std::fmax(smax, v);
+    /* pass 2: weights and the weighted sum of values */
+    double denom = 0.0;
+    for (int32_t e = 0; e < d; ++e) o[e] = 0.0;
+    size_t idx = 0;
+    for (int n = 0; n < nvis; ++n)
+      for (int32_t j = 0; j < chunk_tokens; ++j, ++idx) {
+        const int64_t t = static_cast<int64_t>(vis[n]) * chunk_tokens + j;
+        const double p = std::exp(s[idx] - smax);
+        denom += p;
+        dequant_row(v_codes, v_scales, v_gscale, b, h, t, vrow.data());
+        for (int32_t e = 0; e < d; ++e) o[e] += p * vrow[e];
+      }
+    for (int32_t e = 0; e < d; ++e) out[static_cast<int64_t>(r) * d + e] = o[e] / denom;
+  }
+  return 0;
+}
+
+}  // extern "C"
