@@ -1,0 +1,155 @@
+/*
+ * nvfp4kv.h -- C ABI of libnvfp4kv: an NVFP4 KV cache for chunk-wise autoregressive
+ * video-DiT attention on NVIDIA B200 (sm_100a).
+ *
+ * The method follows the pages on "LongLive-2.0: An NVFP4 Parallel Infrastructure for Long
+ * Video Generation":
+ *  - paper page (paperpeel.com), section 1 "Introduction" and section 3.2 "Parallel KV
+ *    Quantization": the KV cache of the DiT is quantised to NVFP4 and dequantised in
+ *    parallel inside the attention kernel;
+ *  - reading note (yingwang.github.io), "The inference infrastructure": each new chunk's
+ *    K and V are re-quantised at frame-chunk granularity; storage falls from 4*Tc*H*d to
+ *    9/8*Tc*H*d bytes;
+ *  - reading note, "The NVFP4 quantization format", and paper section 2.2 "NVFP4 Training":
+ *    E2M1 elements, one E4M3 scale per 16 elements (largest magnitudes 6 and 448), one FP32
+ *    scale on top; dequantisation is the product of the three;
+ *  - paper section 4.2 "Inference with Multi-Shot Attention Sink": sliding-window attention
+ *    over a KV cache of W chunks plus a permanent global sink, overlaps deduplicated;
+ *    section 2.1: a chunk attends to the preceding clean chunks and to its own tokens.
+ *
+ * Quantisation of one (chunk, head, tensor) with X = chunk_tokens x head_dim bf16 values,
+ * every step one fp32 round-to-nearest-even operation:
+ *    A = max|x|;  g = A / 2688 (0 if A == 0)                 -- FP32 scale, 2688 = 448 * 6
+ *    per token, per 16-element block b along head_dim:
+ *      s_b = E4M3_rn_satfinite(max_b|x| / (6 * g))           (0 if max_b|x| == 0 or g == 0)
+ *      r   = 1 / (s_b * g);  q_i = E2M1_rn_satfinite(x_i * r) (all 0 if s_b == 0 or r is inf)
+ * Dequantisation: x_hat = E2M1(q) * E4M3(s) * g.
+ *
+ * CONVENTIONS (all entry points)
+ *  - Every pointer named "device" is CUDA device memory owned by the caller; the library
+ *    never allocates, frees or keeps device memory, and keeps no state between calls other
+ *    than a per-process cache of driver entry points.
+ *  - Calls are asynchronous on the given CUDA stream (a cudaStream_t passed as void*, NULL
+ *    means the legacy default stream).  The return value reports host-side argument checks
+ *    and launch errors only.  Errors found on the device (a bounded wait that ran out) are
+ *    OR-ed into the cache's device status word; read it with nvfp4kv_read_status().
+ *  - Inputs must be finite.  Non-finite input is a precondition violation, not detected.
+ *  - Supported: head_dim == 128, chunk_tokens even, sm_100a device.
+ */
+#ifndef NVFP4KV_H
+#define NVFP4KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NVFP4KV_OK = 0,
+  NVFP4KV_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misaligned pointer, bad slot */
+  NVFP4KV_ERR_UNSUPPORTED = 2,    /* head_dim != 128, odd chunk_tokens, non-sm_100 device */
+  NVFP4KV_ERR_CUDA = 3,           /* a CUDA runtime or driver call failed */
+  NVFP4KV_ERR_DEVICE_TIMEOUT = 4, /* status bit: a kernel's bounded wait ran out */
+  NVFP4KV_ERR_WORKSPACE = 5       /* workspace pointer null or smaller than required */
+} nvfp4kv_status;
+
+typedef enum { NVFP4KV_OUT_F32 = 0, NVFP4KV_OUT_BF16 = 1 } nvfp4kv_out_dtype;
+
+/* One layer's NVFP4 KV cache.  T = capacity_chunks * chunk_tokens; chunk slot c holds
+ * tokens [c*chunk_tokens, (c+1)*chunk_tokens).  All arrays are device memory:
+ *   k_codes, v_codes   uint8 [batch][heads][T][head_dim/2]   E2M1 pairs, element 2j in the
+ *                                                           low nibble of byte j
+ *   k_scales, v_scales uint8 [batch][heads][T][head_dim/16]  E4M3 block scales
+ *   k_gscale, v_gscale fp32  [batch][heads][capacity_chunks] FP32 scale per chunk
+ *   status             uint32, one word; zero it once before first use
+ * Every array must start on a 16-byte boundary. */
+typedef struct {
+  int32_t batch;
+  int32_t heads;
+  int32_t head_dim;
+  int32_t chunk_tokens;
+  int32_t capacity_chunks;
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  uint8_t* k_scales;
+  uint8_t* v_scales;
+  float* k_gscale;
+  float* v_gscale;
+  uint32_t* status;
+} nvfp4kv_cache;
+
+/* Bytes of each cache array for the given shape (per tensor, K or V): codes, scales and
+ * FP32 scales.  Any output pointer may be NULL.  Returns NVFP4KV_OK or
+ * NVFP4KV_ERR_INVALID_ARG for non-positive sizes or head_dim not a multiple of 16. */
+int nvfp4kv_cache_sizes(int32_t batch, int32_t heads, int32_t head_dim, int32_t chunk_tokens,
+                        int32_t capacity_chunks, size_t* codes_bytes, size_t* scales_bytes,
+                        size_t* gscale_bytes);
+
+/* Workspace bytes nvfp4_kv_quantize and nvfp4_kv_attention need for this cache and a query
+ * chunk of q_tokens tokens (the maximum over both calls; 0 is never returned).  Returns 0
+ * for an invalid cache description. */
+size_t nvfp4kv_workspace_bytes(const nvfp4kv_cache* cache, int32_t q_tokens);
+
+/* Quantise a new frame chunk's K and V and write it into chunk slot `chunk_slot`.
+ *   k_bf16, v_bf16  device bf16, element (b, t, h, e) at [(b*chunk_tokens + t)*token_stride +
+ *                   h*head_dim + e]; 16-byte aligned; token_stride >= heads*head_dim and a
+ *                   multiple of 8
+ *   workspace       device scratch of at least nvfp4kv_workspace_bytes() bytes, 16-byte
+ *                   aligned; its contents on entry do not matter
+ * Writes codes, scales and the FP32 scales of slot `chunk_slot` for every (b, h); nothing
+ * else in the cache is touched.  Bit-for-bit deterministic.
+ * Errors: NVFP4KV_ERR_INVALID_ARG (null, misaligned, slot out of range, bad stride),
+ * NVFP4KV_ERR_UNSUPPORTED, NVFP4KV_ERR_WORKSPACE, NVFP4KV_ERR_CUDA (launch failed). */
+int nvfp4_kv_quantize(const nvfp4kv_cache* cache, int32_t chunk_slot, const void* k_bf16,
+                      const void* v_bf16, int64_t token_stride, void* workspace,
+                      size_t workspace_bytes, void* cuda_stream);
+
+/* Attention of a chunk of bf16 queries over the NVFP4 cache.  The query chunk `q_chunk`
+ * attends to the keys of the visible chunk slots
+ *     V = { c < n_sink_chunks } U { q_chunk - window_chunks < c <= q_chunk },
+ * each slot once (its own chunk included, so it must have been quantised first):
+ *     out_i = sum_j softmax_j(scale * q_i . k_hat_j) v_hat_j    over the keys j of V.
+ *   q_bf16     device bf16, element (b, i, h, e) at [(b*q_tokens + i)*q_token_stride +
+ *              h*head_dim + e]; 16-byte aligned; q_token_stride >= heads*head_dim and a
+ *              multiple of 8
+ *   out        device [batch][q_tokens][heads][head_dim], fp32 or bf16 (out_dtype),
+ *              contiguous, 16-byte aligned
+ *   softmax_scale <= 0 selects 1/sqrt(head_dim)
+ *   workspace  device scratch of at least nvfp4kv_workspace_bytes(cache, q_tokens) bytes
+ * Chunk slots outside V are never read.  Errors as for nvfp4_kv_quantize; window_chunks < 1,
+ * n_sink_chunks < 0 or q_chunk outside [0, capacity) give NVFP4KV_ERR_INVALID_ARG. */
+int nvfp4_kv_attention(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q_tokens,
+                       int64_t q_token_stride, int32_t q_chunk, int32_t n_sink_chunks,
+                       int32_t window_chunks, float softmax_scale, void* out, int32_t out_dtype,
+                       void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* Dequantise chunk slots [first_slot, first_slot + n_slots) of K (which == 0) or V
+ * (which == 1) into device fp32 out[batch][heads][n_slots*chunk_tokens][head_dim]: the
+ * pages' dequantisation step on its own, for tests and diagnostics.  Each value is the
+ * exact E2M1 * E4M3 product times the FP32 scale, rounded once to fp32. */
+int nvfp4_kv_dequantize(const nvfp4kv_cache* cache, int32_t which, int32_t first_slot,
+                        int32_t n_slots, float* out, void* cuda_stream);
+
+/* Diagnostic probe of the device conversions the quantiser uses: for each of the n fp32
+ * values x (device), write the E2M1 code (low nibble; round to nearest even, saturate to
+ * +-6) to e2m1_codes and the E4M3 code (round to nearest even, saturate to +-448) to
+ * e4m3_codes (both device uint8[n]).  Used to compare the hardware conversions with the
+ * format definition over whole ranges of inputs. */
+int nvfp4kv_debug_encode(const float* x, int64_t n, uint8_t* e2m1_codes, uint8_t* e4m3_codes,
+                         void* cuda_stream);
+
+/* Wait for `cuda_stream`, then read the cache's device status word into *out and clear it.
+ * *out == 0 means no device-side error since the last read; otherwise it holds OR-ed
+ * nvfp4kv_status bits (1 << NVFP4KV_ERR_DEVICE_TIMEOUT for a bounded wait that ran out). */
+int nvfp4kv_read_status(const nvfp4kv_cache* cache, void* cuda_stream, uint32_t* out);
+
+/* Static description of a status code.  Never NULL. */
+const char* nvfp4kv_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4KV_H */

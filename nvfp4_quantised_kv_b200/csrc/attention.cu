@@ -1,0 +1,617 @@
+// attention.cu -- chunk attention over the NVFP4 KV cache on sm_100a.
+//
+// Method: "LongLive-2.0" paper page (paperpeel.com), section 1 and section 3.2 "Parallel KV
+// Quantization": the cache stays in NVFP4 and is dequantised in parallel inside the
+// attention kernel; section 4.2 "Inference with Multi-Shot Attention Sink": the query chunk
+// attends to a permanent sink plus a sliding window of chunks (duplicates removed); section
+// 2.1: a chunk sees its own tokens.  Reading note (yingwang.github.io), "The NVFP4
+// quantization format": x_hat = E2M1 * E4M3 * FP32 scale.
+//
+// One CTA owns QT query tiles of 128 rows of one (batch, head) and walks the visible KV
+// tiles (128 keys each; tiles lie inside runs of consecutive visible chunks, so chunks
+// outside the mask are never read).  Warp roles:
+//   softmax warps [0, 4*QT)   one query row per thread, online softmax over TMEM rows
+//   producer warp             TMA: Q tiles (tensor map, 128B swizzle) and packed K/V tiles
+//                             + E4M3 scales (1-D bulk copies) into a ring of smem slots
+//   MMA warp                  TMEM allocation; tcgen05.mma S = Q K^T (both operands in
+//                             smem), O += P V (P from TMEM, V from smem)
+//   dequant warps (4)         E2M1 * E4M3 products, exact in 16 bits, written straight
+//                             into the 128B-swizzled UMMA operand layout: bf16 K (the
+//                             B operand of Q K^T, K-major) and fp16 V (the B operand of
+//                             P V, MN-major)
+// The FP32 scales stay out of the MMAs: g_K(chunk) multiplies S per column, and
+// g_V(chunk) / max g_V multiplies P per column before P is rounded to fp16 (fp16 P and V
+// keep the P V product 8x finer than bf16).  Rows are rescaled lazily: the running max
+// only moves when it grows by more than 2^8.
+//
+// Every mbarrier wait is bounded (%globaltimer); on a time-out the kernel ORs
+// NVFP4KV_ERR_DEVICE_TIMEOUT into the status word, lets in-flight copies and MMAs finish,
+// frees its TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+#include <vector>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace nvfp4kv {
+namespace {
+
+constexpr int BM = 128;  // query rows per tile (TMEM lanes)
+constexpr int BN = 128;  // keys per KV tile
+constexpr int D = kHeadDim;
+constexpr int NST = 2;   // stages of dequantised K / V tiles
+constexpr int NPK = 4;   // slots of packed data (K and V tiles alternate)
+constexpr int PK_CODES = BN * kCodeBytes;               // 8192
+constexpr int PK_BYTES = PK_CODES + BN * kScaleBytes;   // 9216
+constexpr int TILE16 = BN * D * 2;                      // one 128 x 128 16-bit operand tile
+constexpr int HALF16 = TILE16 / 2;                      // 128 rows x 64 elements (128 B rows)
+constexpr int MAX_RUNS = 4;
+
+template <int QT>
+struct Cfg {
+  static constexpr int kSoftmaxWarps = 4 * QT;
+  static constexpr int kProducerWarp = kSoftmaxWarps;
+  static constexpr int kMmaWarp = kSoftmaxWarps + 1;
+  static constexpr int kDequantWarp0 = kSoftmaxWarps + 2;
+  static constexpr int kDequantWarps = 4;
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2 + kDequantWarps);
+  static constexpr uint32_t kTmemCols = QT == 1 ? 256 : 512;
+  // shared memory map (bytes from a 1024-aligned base)
+  static constexpr int oQ = 0;
+  static constexpr int oK = oQ + QT * TILE16;
+  static constexpr int oV = oK + NST * TILE16;
+  static constexpr int oPK = oV + NST * TILE16;
+  static constexpr int oCol = oPK + NPK * PK_BYTES;  // per stage: colK[BN], colV[BN] (fp32)
+  static constexpr int oInfo = oCol + NST * 2 * BN * 4;  // per stage: int4 {n_valid, uniform}
+  static constexpr int oBar = oInfo + NST * 16;
+  // barrier indices
+  static constexpr int bQFull = 0;
+  static constexpr int bPkFull = 1;
+  static constexpr int bPkEmpty = bPkFull + NPK;
+  static constexpr int bKFull = bPkEmpty + NPK;
+  static constexpr int bVFull = bKFull + NST;
+  static constexpr int bKvEmpty = bVFull + NST;
+  static constexpr int bSFull = bKvEmpty + NST;
+  static constexpr int bPFull = bSFull + QT;
+  static constexpr int bODone = bPFull + QT;
+  static constexpr int bDrain = bODone + QT;
+  static constexpr int kNumBars = bDrain + 1;
+  static constexpr int oMisc = oBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag
+  static constexpr int kSmemBytes = oMisc + 16 + 1024;  // + slack for 1024-B alignment
+};
+
+struct AttnParams {
+  const uint8_t* k_codes;
+  const uint8_t* v_codes;
+  const uint8_t* k_scales;
+  const uint8_t* v_scales;
+  const float* k_g;
+  const float* v_g;
+  void* out;
+  uint32_t* status;
+  int64_t T;  // cached tokens per (b, h)
+  int B, H, Lq, Lc, C;
+  int out_bf16;
+  int n_runs;
+  int run_key0[MAX_RUNS];
+  int run_key1[MAX_RUNS];
+  int run_tile0[MAX_RUNS + 1];
+  int n_tiles;
+  float scale_log2;  // softmax scale * log2(e)
+};
+
+// ------------------------------------------------------------------ waits
+__device__ __forceinline__ bool timed_out(uint64_t& t0, int& it) {
+  const uint64_t now = ptx::globaltimer_ns();
+  if (it++ == 0) t0 = now;
+  return now - t0 > kWaitLimitNs;
+}
+
+// Single-thread wait; gives up when another thread aborted or the limit is reached.
+__device__ __forceinline__ bool wait1(uint32_t bar, uint32_t parity, volatile uint32_t* abort, uint32_t* status) {
+  uint64_t t0 = 0;
+  int it = 0;
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (timed_out(t0, it)) {
+      *abort = 1;
+      atomicOr(status, kStatusTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Warp-collective wait: every lane observes the phase; the give-up decision is uniform.
+__device__ __forceinline__ bool waitw(uint32_t bar, uint32_t parity, volatile uint32_t* abort, uint32_t* status) {
+  const int lane = threadIdx.x & 31;
+  uint64_t t0 = 0;
+  int it = 0;
+  while (true) {
+    const bool ok = ptx::mbar_try_wait(bar, parity);
+    if (__all_sync(0xFFFFFFFFu, ok)) return true;
+    uint32_t give_up = 0;
+    if (lane == 0) {
+      if (*abort) {
+        give_up = 1;
+      } else if (timed_out(t0, it)) {
+        *abort = 1;
+        atomicOr(status, kStatusTimeout);
+        give_up = 1;
+      }
+    }
+    if (__shfl_sync(0xFFFFFFFFu, give_up, 0)) return false;
+  }
+}
+
+// Exit-path wait for work that is known to finish (copies or MMAs already issued).
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, uint32_t* status) {
+  uint64_t t0 = 0;
+  int it = 0;
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if (timed_out(t0, it)) {
+      atomicOr(status, kStatusTimeout);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ void tile_keys(const AttnParams& p, int j, int& key0, int& n) {
+  int r = 0;
+  while (r + 1 < p.n_runs && j >= p.run_tile0[r + 1]) ++r;
+  key0 = p.run_key0[r] + (j - p.run_tile0[r]) * BN;
+  n = min(BN, p.run_key1[r] - key0);
+}
+
+__device__ __forceinline__ float max_visible_gv(const AttnParams& p, int64_t bh) {
+  float m = 0.0f;
+  for (int r = 0; r < p.n_runs; ++r)
+    for (int c = p.run_key0[r] / p.Lc; c < p.run_key1[r] / p.Lc; ++c)
+      m = fmaxf(m, p.v_g[bh * p.C + c]);
+  return m > 0.0f ? m : 1.0f;
+}
+
+// Dequantise one packed tile (codes + E4M3 scales of BN keys) into a 128B-swizzled
+// [key][d] operand tile of 16-bit values.  Thread dt of 128 handles 16 groups of 8
+// elements; a warp covers two keys (4 x 128 B rows) per step, conflict-free.
+template <bool kBF16>
+__device__ __forceinline__ void dequant_tile(const uint8_t* pk, uint8_t* dst, int n, int dt) {
+#pragma unroll 4
+  for (int it = 0; it < 16; ++it) {
+    const int job = it * 128 + dt;
+    const int key = job >> 4;
+    const int c16 = job & 15;
+    uint4 o = make_uint4(0, 0, 0, 0);
+    if (key < n) {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(pk + key * kCodeBytes + c16 * 4);
+      const uint32_t sb = pk[PK_CODES + key * kScaleBytes + (c16 >> 1)];
+      uint32_t h[4];
+      ptx::e2m1x8_to_f16x8(w, h);
+      const uint32_t s2 = ptx::e4m3_to_f16x2_bcast(sb);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        h[i] = ptx::hmul2_u32(h[i], s2);
+        if (kBF16) h[i] = ptx::f16x2_to_bf16x2(h[i]);
+      }
+      o = make_uint4(h[0], h[1], h[2], h[3]);
+    }
+    const int off = (c16 >> 3) * HALF16 + key * 128 + (((c16 & 7) ^ (key & 7)) << 4);
+    *reinterpret_cast<uint4*>(dst + off) = o;
+  }
+}
+
+template <int QT>
+__global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
+    attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ AttnParams p) {
+  using C = Cfg<QT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int m0 = blockIdx.x * (BM * QT);
+  const int64_t bh = static_cast<int64_t>(b) * p.H + h;
+
+  const uint32_t sbase = ptx::smem_u32(smem);
+  auto bar = [&](int i) { return sbase + C::oBar + 8 * i; };
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::oMisc);
+  volatile uint32_t* abort_flag = misc + 1;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar(C::bQFull), 1);
+    for (int i = 0; i < NPK; ++i) {
+      ptx::mbar_init(bar(C::bPkFull + i), 1);
+      ptx::mbar_init(bar(C::bPkEmpty + i), C::kDequantWarps);
+    }
+    for (int i = 0; i < NST; ++i) {
+      ptx::mbar_init(bar(C::bKFull + i), C::kDequantWarps);
+      ptx::mbar_init(bar(C::bVFull + i), C::kDequantWarps);
+      ptx::mbar_init(bar(C::bKvEmpty + i), 1);
+    }
+    for (int q = 0; q < QT; ++q) {
+      ptx::mbar_init(bar(C::bSFull + q), 1);
+      ptx::mbar_init(bar(C::bPFull + q), 4);
+      ptx::mbar_init(bar(C::bODone + q), 1);
+    }
+    ptx::mbar_init(bar(C::bDrain), 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::fence_proxy_async_smem();
+  }
+  if (warp == C::kMmaWarp) {
+    ptx::tmem_alloc(sbase + C::oMisc, C::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp < C::kSoftmaxWarps) {
+    // ============================================================ softmax + epilogue
+    const int qt = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + qt * BN;
+    const uint32_t tO = tmem + lane_off + QT * BN + qt * D;
+    const float gv_ref = max_visible_gv(p, bh);
+    float m_run = -INFINITY, l_run = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < p.n_tiles && ok; ++j) {
+      const int st = j % NST;
+      ok = waitw(bar(C::bSFull + qt), j & 1, abort_flag, p.status) &&
+           waitw(bar(C::bKFull + st), (j / NST) & 1, abort_flag, p.status);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      float x[BN];
+      {
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          ptx::tmem_ld32(tS + 32 * c, r);
+          ptx::tc_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(r[i]);
+        }
+      }
+      const int4 info = *reinterpret_cast<const int4*>(smem + C::oInfo + 16 * st);
+      const float* colK = reinterpret_cast<const float*>(smem + C::oCol + st * 2 * BN * 4);
+      const float* colV = colK + BN;
+      float mx = -INFINITY;
+      if (info.y) {
+        const float ck = colK[0];
+#pragma unroll
+        for (int i = 0; i < BN; ++i) {
+          x[i] *= ck;
+          mx = fmaxf(mx, x[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < BN; ++i) {
+          x[i] = (i < info.x) ? x[i] * colK[i] : -INFINITY;
+          mx = fmaxf(mx, x[i]);
+        }
+      }
+      if (mx > m_run + 8.0f) {
+        const float alpha = ptx::ex2(m_run - mx);
+        l_run *= alpha;
+        m_run = mx;
+        if (j > 0) {
+          ok = waitw(bar(C::bODone + qt), (j - 1) & 1, abort_flag, p.status);
+          if (!ok) break;
+          ptx::tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(tO + 32 * c, r);
+            ptx::tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            ptx::tmem_st32(tO + 32 * c, r);
+          }
+        }
+      }
+      // P~ = 2^(x - m) * g_V(chunk) / max g_V, rounded to fp16 pairs, written over S's first
+      // 64 TMEM columns (S is fully in registers by now).
+      float lsum = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        if (info.y) {
+          const float cv = colV[0];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = ptx::ex2(x[64 * c + 2 * i] - m_run);
+            const float p1 = ptx::ex2(x[64 * c + 2 * i + 1] - m_run);
+            lsum += p0 + p1;
+            r[i] = ptx::f32x2_to_f16x2(p0 * cv, p1 * cv);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = ptx::ex2(x[64 * c + 2 * i] - m_run);
+            const float p1 = ptx::ex2(x[64 * c + 2 * i + 1] - m_run);
+            lsum += p0 + p1;
+            r[i] = ptx::f32x2_to_f16x2(p0 * colV[64 * c + 2 * i], p1 * colV[64 * c + 2 * i + 1]);
+          }
+        }
+        ptx::tmem_st32(tS + 32 * c, r);
+      }
+      l_run += lsum;
+      ptx::tc_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(C::bPFull + qt));
+    }
+    if (ok && p.n_tiles > 0) {
+      ok = waitw(bar(C::bODone + qt), (p.n_tiles - 1) & 1, abort_flag, p.status);
+      if (ok) {
+        ptx::tc_fence_after();
+        const float inv = gv_ref / l_run;
+        const int qrow = m0 + qt * BM + row;
+        const bool store = qrow < p.Lq;
+        const int64_t obase = ((static_cast<int64_t>(b) * p.Lq + qrow) * p.H + h) * D;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tO + 32 * c, r);
+          ptx::tc_wait_ld();
+          if (store) {
+            if (p.out_bf16) {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + obase + 32 * c);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                uint32_t w[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(r[8 * i + 2 * k]) * inv,
+                                                            __uint_as_float(r[8 * i + 2 * k + 1]) * inv);
+                  w[k] = *reinterpret_cast<uint32_t*>(&v2);
+                }
+                dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            } else {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + 32 * c);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
+                                     __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv);
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == C::kProducerWarp) {
+    // ============================================================ TMA producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmap_q);
+      ptx::mbar_arrive_expect_tx(bar(C::bQFull), QT * TILE16);
+      for (int q = 0; q < QT; ++q)
+        for (int half = 0; half < 2; ++half)
+          ptx::tma_load_4d(sbase + C::oQ + q * TILE16 + half * HALF16, &tmap_q, half * 64, h,
+                           m0 + q * BM, b, bar(C::bQFull));
+      const uint8_t* kc = p.k_codes + bh * p.T * kCodeBytes;
+      const uint8_t* vc = p.v_codes + bh * p.T * kCodeBytes;
+      const uint8_t* ks = p.k_scales + bh * p.T * kScaleBytes;
+      const uint8_t* vs = p.v_scales + bh * p.T * kScaleBytes;
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < p.n_tiles && ok; ++j) {
+        int key0, n;
+        tile_keys(p, j, key0, n);
+        for (int t = 0; t < 2; ++t) {
+          const int pk = 2 * j + t;
+          const int slot = pk % NPK;
+          ok = wait1(bar(C::bPkEmpty + slot), ((pk / NPK) & 1) ^ 1, abort_flag, p.status);
+          if (!ok) break;
+          const uint32_t dst = sbase + C::oPK + slot * PK_BYTES;
+          ptx::mbar_arrive_expect_tx(bar(C::bPkFull + slot), n * (kCodeBytes + kScaleBytes));
+          ptx::bulk_g2s(dst, (t == 0 ? kc : vc) + static_cast<int64_t>(key0) * kCodeBytes,
+                        n * kCodeBytes, bar(C::bPkFull + slot));
+          ptx::bulk_g2s(dst + PK_CODES, (t == 0 ? ks : vs) + static_cast<int64_t>(key0) * kScaleBytes,
+                        n * kScaleBytes, bar(C::bPkFull + slot));
+          issued = pk + 1;
+        }
+      }
+      if (!ok) {  // let every copy already issued land before the CTA can exit
+        wait_drain(bar(C::bQFull), 0, p.status);
+        for (int pk = std::max(0, issued - NPK); pk < issued; ++pk)
+          wait_drain(bar(C::bPkFull + pk % NPK), (pk / NPK) & 1, p.status);
+      }
+    }
+    __syncwarp();
+  } else if (warp == C::kMmaWarp) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      // kind::f16 instruction descriptors: fp32 accumulate; M = 128; N = 128.
+      constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) |  // bf16 x bf16, both K-major
+                                    (static_cast<uint32_t>(BN >> 3) << 17) |
+                                    (static_cast<uint32_t>(BM >> 4) << 24);
+      constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) |  // fp16 x fp16, B (V) MN-major
+                                    (static_cast<uint32_t>(D >> 3) << 17) |
+                                    (static_cast<uint32_t>(BM >> 4) << 24);
+      bool ok = wait1(bar(C::bQFull), 0, abort_flag, p.status);
+      for (int j = 0; j < p.n_tiles && ok; ++j) {
+        const int st = j % NST;
+        ok = wait1(bar(C::bKFull + st), (j / NST) & 1, abort_flag, p.status);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const uint32_t sK = sbase + C::oK + st * TILE16;
+        for (int q = 0; q < QT; ++q) {
+          const uint32_t sQ = sbase + C::oQ + q * TILE16;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * HALF16 + (kk & 3) * 32;
+            ptx::mma_ss(tmem + q * BN, ptx::smem_desc_sw128(sQ + koff, 16, 1024),
+                        ptx::smem_desc_sw128(sK + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+          }
+          ptx::mma_commit(bar(C::bSFull + q));
+        }
+        const uint32_t sV = sbase + C::oV + st * TILE16;
+        for (int q = 0; q < QT && ok; ++q) {
+          ok = wait1(bar(C::bPFull + q), j & 1, abort_flag, p.status);
+          if (ok && q == 0) ok = wait1(bar(C::bVFull + st), (j / NST) & 1, abort_flag, p.status);
+          if (!ok) break;
+          ptx::tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            ptx::mma_ts(tmem + QT * BN + q * D, tmem + q * BN + kk * 8,
+                        ptx::smem_desc_sw128(sV + kk * 2048, HALF16, 1024), kIdescPV,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          ptx::mma_commit(bar(C::bODone + q));
+        }
+        if (ok) ptx::mma_commit(bar(C::bKvEmpty + st));
+      }
+      // every MMA issued so far completes before the drain barrier's phase 0
+      ptx::mma_commit(bar(C::bDrain));
+      wait_drain(bar(C::bDrain), 0, p.status);
+    }
+    __syncwarp();
+  } else {
+    // ============================================================ dequant warps
+    const int dt = threadIdx.x - C::kDequantWarp0 * 32;
+    const float inv_gv = 1.0f / max_visible_gv(p, bh);
+    bool ok = true;
+    for (int j = 0; j < p.n_tiles && ok; ++j) {
+      const int st = j % NST;
+      if (j >= NST) ok = waitw(bar(C::bKvEmpty + st), ((j / NST) - 1) & 1, abort_flag, p.status);
+      if (!ok) break;
+      int key0, n;
+      tile_keys(p, j, key0, n);
+      for (int t = 0; t < 2 && ok; ++t) {
+        const int pk = 2 * j + t;
+        const int slot = pk % NPK;
+        ok = waitw(bar(C::bPkFull + slot), (pk / NPK) & 1, abort_flag, p.status);
+        if (!ok) break;
+        const uint8_t* src = smem + C::oPK + slot * PK_BYTES;
+        if (t == 0) {
+          dequant_tile<true>(src, smem + C::oK + st * TILE16, n, dt);
+          float* colK = reinterpret_cast<float*>(smem + C::oCol + st * 2 * BN * 4);
+          const bool valid = dt < n;
+          const int c = valid ? (key0 + dt) / p.Lc : 0;
+          colK[dt] = valid ? p.k_g[bh * p.C + c] * p.scale_log2 : 0.0f;
+          colK[BN + dt] = valid ? p.v_g[bh * p.C + c] * inv_gv : 0.0f;
+          if (dt == 0) {
+            const int uniform = (n == BN) && (key0 / p.Lc == (key0 + BN - 1) / p.Lc);
+            *reinterpret_cast<int4*>(smem + C::oInfo + 16 * st) = make_int4(n, uniform, 0, 0);
+          }
+        } else {
+          dequant_tile<false>(src, smem + C::oV + st * TILE16, n, dt);
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive(bar(C::bPkEmpty + slot));
+          ptx::mbar_arrive(bar(t == 0 ? C::bKFull + st : C::bVFull + st));
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == C::kMmaWarp) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+template <int QT>
+cudaError_t launch(const CUtensorMap& tm, const AttnParams& prm, cudaStream_t stream) {
+  using C = Cfg<QT>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(attention_kernel<QT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const dim3 grid((prm.Lq + BM * QT - 1) / (BM * QT), prm.H, prm.B);
+  attention_kernel<QT><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tm, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t attention_workspace_bytes(const nvfp4kv_cache&, int) { return 0; }
+
+int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, int64_t q_stride,
+                     int q_chunk, int n_sink, int window, float softmax_scale, void* out,
+                     int out_dtype, void*, size_t, cudaStream_t stream) {
+  AttnParams prm{};
+  prm.k_codes = c.k_codes;
+  prm.v_codes = c.v_codes;
+  prm.k_scales = c.k_scales;
+  prm.v_scales = c.v_scales;
+  prm.k_g = c.k_gscale;
+  prm.v_g = c.v_gscale;
+  prm.out = out;
+  prm.status = c.status;
+  prm.T = static_cast<int64_t>(c.capacity_chunks) * c.chunk_tokens;
+  prm.B = c.batch;
+  prm.H = c.heads;
+  prm.Lq = q_tokens;
+  prm.Lc = c.chunk_tokens;
+  prm.C = c.capacity_chunks;
+  prm.out_bf16 = out_dtype == NVFP4KV_OUT_BF16 ? 1 : 0;
+  const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(D));
+  prm.scale_log2 = scale * 1.4426950408889634f;
+
+  // Visible chunk slots {c < n_sink} U {q_chunk - window < c <= q_chunk}, merged into runs of
+  // consecutive slots; KV tiles never cross a run boundary.
+  std::vector<int> vis;
+  for (int ch = 0; ch < c.capacity_chunks; ++ch)
+    if (ch < n_sink || (ch > q_chunk - window && ch <= q_chunk)) vis.push_back(ch);
+  prm.n_runs = 0;
+  prm.run_tile0[0] = 0;
+  for (size_t i = 0; i < vis.size();) {
+    size_t k = i;
+    while (k + 1 < vis.size() && vis[k + 1] == vis[k] + 1) ++k;
+    if (prm.n_runs == MAX_RUNS) return NVFP4KV_ERR_UNSUPPORTED;
+    const int r = prm.n_runs++;
+    prm.run_key0[r] = vis[i] * c.chunk_tokens;
+    prm.run_key1[r] = (vis[k] + 1) * c.chunk_tokens;
+    prm.run_tile0[r + 1] = prm.run_tile0[r] + (prm.run_key1[r] - prm.run_key0[r] + BN - 1) / BN;
+    i = k + 1;
+  }
+  prm.n_tiles = prm.run_tile0[prm.n_runs];
+
+  PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
+  if (!encode) return NVFP4KV_ERR_CUDA;
+  CUtensorMap tm;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(c.heads),
+                              static_cast<cuuint64_t>(q_tokens), static_cast<cuuint64_t>(c.batch)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(q_stride) * 2,
+                                 static_cast<cuuint64_t>(q_tokens) * q_stride * 2};
+  const cuuint32_t box[4] = {64, 1, BM, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult cr = encode(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(q), dims,
+                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return NVFP4KV_ERR_CUDA;
+  const cudaError_t e = launch<1>(tm, prm, stream);
+  return e == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
+}
+
+}  // namespace nvfp4kv

@@ -1,0 +1,40 @@
+// internal.h -- declarations shared by the library's translation units (not installed).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/nvfp4kv.h"
+
+namespace nvfp4kv {
+
+constexpr int kHeadDim = 128;
+constexpr int kBlock = 16;                    // elements per E4M3 block scale
+constexpr int kCodeBytes = kHeadDim / 2;      // 64 bytes of E2M1 codes per token and head
+constexpr int kScaleBytes = kHeadDim / kBlock;  // 8 E4M3 scale bytes per token and head
+constexpr uint32_t kStatusTimeout = 1u << NVFP4KV_ERR_DEVICE_TIMEOUT;
+
+// Bounded-wait limit for every in-kernel wait (nanoseconds of %globaltimer).
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+
+// ---- quantiser (quantize.cu)
+// Number of amax partial slots per (b, h, tensor) and the workspace bytes they need.
+int quantize_parts(int batch, int heads, int chunk_tokens);
+size_t quantize_workspace_bytes(int batch, int heads, int chunk_tokens);
+cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
+                            int64_t token_stride, void* workspace, cudaStream_t stream);
+
+// ---- attention (attention.cu)
+size_t attention_workspace_bytes(const nvfp4kv_cache& c, int q_tokens);
+int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, int64_t q_stride,
+                     int q_chunk, int n_sink, int window, float softmax_scale, void* out,
+                     int out_dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+// ---- diagnostics (dequantize.cu)
+cudaError_t launch_dequantize(const nvfp4kv_cache& c, int which, int first_slot, int n_slots,
+                              float* out, cudaStream_t stream);
+cudaError_t launch_encode_probe(const float* x, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
+                                cudaStream_t stream);
+
+}  // namespace nvfp4kv

@@ -30,6 +30,10 @@ def lib() -> ctypes.CDLL:
         L.oracle_e4m3_decode.restype = ctypes.c_double
         L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        for name in ("oracle_e2m1_encode_array", "oracle_e4m3_encode_array"):
+            fn = getattr(L, name)
+            fn.restype = None
+            fn.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
         L.oracle_quantize_chunk.restype = ctypes.c_int
         L.oracle_quantize_chunk.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
                                             ctypes.c_int32, ctypes.c_int32, ctypes.c_int64,
@@ -69,6 +73,20 @@ def e4m3_decode(code: int) -> float:
 
 def e4m3_encode(v: float) -> int:
     return lib().oracle_e4m3_encode(v)
+
+
+def e2m1_encode_array(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.zeros(x.shape, np.uint8)
+    lib().oracle_e2m1_encode_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def e4m3_encode_array(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.zeros(x.shape, np.uint8)
+    lib().oracle_e4m3_encode_array(_ptr(x), x.size, _ptr(out))
+    return out
 
 
 def quantize_chunk(x_bf16: np.ndarray, token_stride: int | None = None):

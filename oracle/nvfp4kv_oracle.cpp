@@ -111,6 +111,16 @@ uint8_t oracle_e4m3_encode(float v) {
                                                             e4m3_magnitude));
 }
 
+void oracle_e2m1_encode_array(const float* x, int64_t n, uint8_t* out) {
+  IeeeMode ieee;
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_e2m1_encode(x[i]);
+}
+
+void oracle_e4m3_encode_array(const float* x, int64_t n, uint8_t* out) {
+  IeeeMode ieee;
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_encode(x[i]);
+}
+
 int oracle_quantize_chunk(const uint16_t* x, int32_t B, int32_t L, int32_t H, int32_t d,
                           int64_t token_stride, uint8_t* codes, uint8_t* scales, float* gscale) {
   if (!x || !codes || !scales || !gscale || B <= 0 || L <= 0 || H <= 0 || d <= 0 || d % 16 != 0 ||
@@ -229,39 +239,47 @@ int oracle_attention_rows(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, i
     }
   };
 
-  std::vector<double> qrow(static_cast<size_t>(d)), krow(static_cast<size_t>(d)),
-      vrow(static_cast<size_t>(d)), o(static_cast<size_t>(d));
-  std::vector<double> s;
+  /* The visible keys of one (b, h), dequantised once and reused for every requested row of
+   * that (b, h); the arithmetic per row is unchanged. */
+  std::vector<int64_t> keys;
+  for (int n = 0; n < nvis; ++n)
+    for (int32_t j = 0; j < chunk_tokens; ++j)
+      keys.push_back(static_cast<int64_t>(vis[n]) * chunk_tokens + j);
+  const size_t nk = keys.size();
+  std::vector<double> khat(nk * d), vhat(nk * d);
+  int32_t cached_b = -1, cached_h = -1;
+
+  std::vector<double> qrow(static_cast<size_t>(d)), o(static_cast<size_t>(d)), s(nk);
   for (int32_t r = 0; r < n_rows; ++r) {
     const int32_t b = rows[3 * r + 0], h = rows[3 * r + 1], i = rows[3 * r + 2];
     if (b < 0 || b >= B || h < 0 || h >= H || i < 0 || i >= Lq) return -1;
+    if (b != cached_b || h != cached_h) {
+      for (size_t k = 0; k < nk; ++k) {
+        dequant_row(k_codes, k_scales, k_gscale, b, h, keys[k], &khat[k * d]);
+        dequant_row(v_codes, v_scales, v_gscale, b, h, keys[k], &vhat[k * d]);
+      }
+      cached_b = b;
+      cached_h = h;
+    }
     for (int32_t e = 0; e < d; ++e)
       qrow[e] = bf16_bits_to_float(q[(static_cast<int64_t>(b) * Lq + i) * q_token_stride +
                                      static_cast<int64_t>(h) * d + e]);
     /* pass 1: logits over every visible key */
-    s.clear();
-    for (int n = 0; n < nvis; ++n)
-      for (int32_t j = 0; j < chunk_tokens; ++j) {
-        const int64_t t = static_cast<int64_t>(vis[n]) * chunk_tokens + j;
-        dequant_row(k_codes, k_scales, k_gscale, b, h, t, krow.data());
-        double dot = 0.0;
-        for (int32_t e = 0; e < d; ++e) dot += qrow[e] * krow[e];
-        s.push_back(sigma * dot);
-      }
     double smax = -std::numeric_limits<double>::infinity();
-    for (double v : s) smax = std::fmax(smax, v);
+    for (size_t k = 0; k < nk; ++k) {
+      double dot = 0.0;
+      for (int32_t e = 0; e < d; ++e) dot += qrow[e] * khat[k * d + e];
+      s[k] = sigma * dot;
+      smax = std::fmax(smax, s[k]);
+    }
     /* pass 2: weights and the weighted sum of values */
     double denom = 0.0;
     for (int32_t e = 0; e < d; ++e) o[e] = 0.0;
-    size_t idx = 0;
-    for (int n = 0; n < nvis; ++n)
-      for (int32_t j = 0; j < chunk_tokens; ++j, ++idx) {
-        const int64_t t = static_cast<int64_t>(vis[n]) * chunk_tokens + j;
-        const double p = std::exp(s[idx] - smax);
-        denom += p;
-        dequant_row(v_codes, v_scales, v_gscale, b, h, t, vrow.data());
-        for (int32_t e = 0; e < d; ++e) o[e] += p * vrow[e];
-      }
+    for (size_t k = 0; k < nk; ++k) {
+      const double p = std::exp(s[k] - smax);
+      denom += p;
+      for (int32_t e = 0; e < d; ++e) o[e] += p * vhat[k * d + e];
+    }
     for (int32_t e = 0; e < d; ++e) out[static_cast<int64_t>(r) * d + e] = o[e] / denom;
   }
   return 0;

@@ -44,6 +44,10 @@ uint8_t oracle_e2m1_encode(float v);      /* round to nearest, ties to even code
 double  oracle_e4m3_decode(uint8_t code); /* NaN for 0x7F / 0xFF */
 uint8_t oracle_e4m3_encode(float v);      /* round to nearest, ties to even code, clamp to +-448 */
 
+/* Element-wise encoders over arrays (out[i] = encode(x[i])), for sweeping conversions. */
+void oracle_e2m1_encode_array(const float* x, int64_t n, uint8_t* out);
+void oracle_e4m3_encode_array(const float* x, int64_t n, uint8_t* out);
+
 /* Quantise one chunk of one tensor (K or V) for every (b, h).
  * x       : bf16 bit patterns, element (b, t, h, i) at x[(b*L + t)*token_stride + h*d + i]
  * codes   : [B][H][L][d/2], scales: [B][H][L][d/16], gscale: [B][H]

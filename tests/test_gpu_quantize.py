@@ -1,0 +1,114 @@
+"""GPU parity of the quantiser and of the dequantisation step: codes, E4M3 scales and FP32
+scales bit-identical to the oracle on the same seeded inputs; dequantised values equal to
+the oracle's exact fp64 values rounded once to fp32."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import oracle
+from nvfp4_quantised_kv_b200 import KVCache, debug_encode, synthetic
+from tests import special_chunks as sc
+from tests.gpu_util import assert_cache_equal, dev_bf16, make_caches
+
+pytestmark = pytest.mark.gpu
+
+
+def _sweep_values():
+    """Every finite bf16 value, dense neighbourhoods of every E2M1 / E4M3 rounding boundary
+    (+-512 ulps), and random finite fp32 bit patterns."""
+    rng = np.random.default_rng(123)
+    bf = (np.arange(65536, dtype=np.uint32) << 16).view(np.float32)
+    vals = [bf[np.isfinite(bf)]]
+    e2 = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0]
+    e4 = sorted(set(sc.e4m3_positive_values()))
+    e4_mid = [(a + b) / 2 for a, b in zip([0.0] + e4[:-1], e4)] + [448.0, 464.0]
+    centers = np.array(e2 + e4_mid, np.float32)
+    off = np.arange(-512, 513, dtype=np.int64)
+    for c in centers:
+        u = np.int64(np.float32(c).view(np.uint32)) + off
+        u = u[(u > 0) & (u < 0x7F800000)].astype(np.uint32)
+        v = u.view(np.float32)
+        vals += [v, -v]
+    r = rng.integers(0, 2 ** 32, size=1 << 22, dtype=np.uint64).astype(np.uint32).view(np.float32)
+    vals.append(r[np.isfinite(r)])
+    return np.concatenate(vals)
+
+
+def test_device_conversions_match_the_format_definition():
+    import torch
+    x = _sweep_values()
+    e2, e4 = debug_encode(torch.from_numpy(x).cuda())
+    e2, e4 = e2.cpu().numpy(), e4.cpu().numpy()
+    want2 = oracle.e2m1_encode_array(x)
+    want4 = oracle.e4m3_encode_array(x)
+    bad2 = np.nonzero(e2 != want2)[0]
+    bad4 = np.nonzero(e4 != want4)[0]
+    assert bad2.size == 0, (x[bad2[:8]], e2[bad2[:8]], want2[bad2[:8]])
+    assert bad4.size == 0, (x[bad4[:8]], e4[bad4[:8]], want4[bad4[:8]])
+
+
+@pytest.mark.parametrize("key,slots", [("tiny", [0, 1, 2, 3]), ("1.3b", [0, 3]), ("5b", [1, 6]),
+                                       ("fewstep", [6]), ("rollout", [39])])
+def test_quantize_matches_oracle_bit_for_bit(key, slots):
+    w = synthetic.WORKLOADS[key]
+    cache, ocache = make_caches(w, slots)
+    assert_cache_equal(cache, ocache, slots)
+    assert cache.read_status() == 0
+
+
+@pytest.mark.parametrize("name", ["fixed0", "fixed-20", "fixed17", "fixed-100", "ties0", "ties-9",
+                                  "underflow", "tiny_scale"])
+def test_special_chunks_match_oracle(name):
+    chunk = {"fixed0": lambda: sc.fixed_point_chunk(0), "fixed-20": lambda: sc.fixed_point_chunk(-20),
+             "fixed17": lambda: sc.fixed_point_chunk(17), "fixed-100": lambda: sc.fixed_point_chunk(-100),
+             "ties0": lambda: sc.tie_chunk(0), "ties-9": lambda: sc.tie_chunk(-9),
+             "underflow": sc.underflow_chunk, "tiny_scale": sc.tiny_scale_chunk}[name]()
+    chunk = sc.pad_tokens(chunk)
+    L = chunk.shape[1]
+    cache = KVCache(1, 1, L, 2)
+    ocache = oracle.Cache(1, 1, 128, L, 2)
+    neg = chunk ^ np.uint16(0x8000)  # V gets the negated chunk
+    cache.quantize(1, dev_bf16(chunk), dev_bf16(neg))
+    ocache.append(1, chunk, neg)
+    assert_cache_equal(cache, ocache, [1])
+    # the slot not written stays untouched
+    assert int(cache.k_codes[:, :, :L].abs().sum()) == 0
+
+
+def test_token_stride_fused_qkv_layout():
+    import torch
+    w = dataclasses.replace(synthetic.WORKLOADS["tiny"], heads=3, chunk_tokens=96, batch=2)
+    k, v = synthetic.chunk_kv(w, 0)
+    qkv = torch.zeros(w.batch, w.chunk_tokens, 3, w.heads, 128, dtype=torch.bfloat16, device="cuda")
+    qkv[:, :, 1] = dev_bf16(k)
+    qkv[:, :, 2] = dev_bf16(v)
+    cache = KVCache(w.batch, w.heads, w.chunk_tokens, 2)
+    cache.quantize(1, qkv[:, :, 1], qkv[:, :, 2])
+    ocache = oracle.Cache(w.batch, w.heads, 128, w.chunk_tokens, 2)
+    ocache.append(1, k, v)
+    assert_cache_equal(cache, ocache, [1])
+
+
+def test_dequantize_matches_oracle_exact_values():
+    w = synthetic.WORKLOADS["tiny"]
+    cache, ocache = make_caches(w, [0, 1, 2, 3])
+    for which in ("k", "v"):
+        got = cache.dequantize(which).cpu().numpy()
+        want = ocache.dequantize(which).astype(np.float32)
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32)), which
+    got = cache.dequantize("v", first_slot=2, n_slots=2).cpu().numpy()
+    want = ocache.dequantize("v")[:, :, 2 * w.chunk_tokens:].astype(np.float32)
+    assert np.array_equal(got, want)
+
+
+def test_quantize_is_deterministic():
+    w = synthetic.WORKLOADS["5b"]
+    cache, _ = make_caches(w, [])
+    k, v = synthetic.chunk_kv(w, 2)
+    kd, vd = dev_bf16(k), dev_bf16(v)
+    cache.quantize(2, kd, vd)
+    first = [t.clone() for t in (cache.k_codes, cache.v_scales, cache.k_gscale)]
+    cache.quantize(2, kd, vd)
+    for a, b in zip(first, (cache.k_codes, cache.v_scales, cache.k_gscale)):
+        assert bool((a == b).all())
