@@ -283,67 +283,92 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       const int4 info = *reinterpret_cast<const int4*>(smem + C::oInfo + 16 * st);
       const float* colK = reinterpret_cast<const float*>(smem + C::oCol + st * 2 * BN * 4);
       const float* colV = colK + BN;
-      float mx = -INFINITY;
+      // Row maximum of the log2-domain logits x = S * g_K(chunk) * scale * log2(e).  In a
+      // tile inside one chunk (info.y) x stays unscaled here: g_K >= 0 scales the maximum.
+      float mx;
       if (info.y) {
-        const float ck = colK[0];
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int i = 0; i < BN; ++i) {
-          x[i] *= ck;
-          mx = fmaxf(mx, x[i]);
-        }
+        for (int i = 0; i < BN; ++i) m4[i & 3] = fmaxf(m4[i & 3], x[i]);
+        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * colK[0];
       } else {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int i = 0; i < BN; ++i) {
           x[i] = (i < info.x) ? x[i] * colK[i] : -INFINITY;
-          mx = fmaxf(mx, x[i]);
+          m4[i & 3] = fmaxf(m4[i & 3], x[i]);
         }
+        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
-      if (mx > m_run + 8.0f) {
-        const float alpha = ptx::ex2(m_run - mx);
+      // Lazy rescale: a row moves its running max only when it grew by more than 2^8.  The
+      // O rescale uses warp-collective TMEM accesses, so it runs for the whole warp when any
+      // row of the warp moved (alpha = 1 for the rows that did not).
+      const bool moved = mx > m_run + 8.0f;
+      float alpha = 1.0f;
+      if (moved) {
+        alpha = ptx::ex2(m_run - mx);
         l_run *= alpha;
         m_run = mx;
-        if (j > 0) {
-          ok = waitw(bar(C::bODone + qt), (j - 1) & 1, abort_flag, p.status);
-          if (!ok) break;
-          ptx::tc_fence_after();
+      }
+      if (j > 0 && __any_sync(0xFFFFFFFFu, moved)) {
+        ok = waitw(bar(C::bODone + qt), (j - 1) & 1, abort_flag, p.status);
+        if (!ok) break;
+        ptx::tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tO + 32 * c, r);
-            ptx::tc_wait_ld();
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tO + 32 * c, r);
+          ptx::tc_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            ptx::tmem_st32(tO + 32 * c, r);
-          }
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          ptx::tmem_st32(tO + 32 * c, r);
         }
       }
-      // P~ = 2^(x - m) * g_V(chunk) / max g_V, rounded to fp16 pairs, written over S's first
-      // 64 TMEM columns (S is fully in registers by now).
-      float lsum = 0.0f;
+      // P~ = 2^(x - m) * cv, cv = g_V(chunk) / max g_V, rounded to fp16 pairs and written over
+      // S's first 64 TMEM columns (S is fully in registers by now).  The row sum l adds the
+      // same rounded values divided by cv, so the rounding of P~ largely cancels in O / l.
+      // A key of an all-zero V chunk (cv = 0) contributes 0 to O and its p to l.
+      float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (info.y) {
+        const float ck = colK[0], cv = colV[0];
+        const float mneg = (cv > 0.0f ? log2f(cv) : 0.0f) - m_run;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
-        if (info.y) {
-          const float cv = colV[0];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float p0 = ptx::ex2(x[64 * c + 2 * i] - m_run);
-            const float p1 = ptx::ex2(x[64 * c + 2 * i + 1] - m_run);
-            lsum += p0 + p1;
-            r[i] = ptx::f32x2_to_f16x2(p0 * cv, p1 * cv);
-          }
-        } else {
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float p0 = ptx::ex2(x[64 * c + 2 * i] - m_run);
-            const float p1 = ptx::ex2(x[64 * c + 2 * i + 1] - m_run);
-            lsum += p0 + p1;
-            r[i] = ptx::f32x2_to_f16x2(p0 * colV[64 * c + 2 * i], p1 * colV[64 * c + 2 * i + 1]);
+            const float p0 = ptx::ex2(fmaf(x[64 * c + 2 * i], ck, mneg));
+            const float p1 = ptx::ex2(fmaf(x[64 * c + 2 * i + 1], ck, mneg));
+            if (cv > 0.0f) {
+              r[i] = ptx::f32x2_to_f16x2(p0, p1);
+              ls[i & 3] = ptx::add_f16x2_f32(ls[i & 3], r[i]);
+            } else {
+              r[i] = 0u;
+              ls[i & 3] += p0 + p1;
+            }
           }
+          ptx::tmem_st32(tS + 32 * c, r);
         }
-        ptx::tmem_st32(tS + 32 * c, r);
+        const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        l_run += cv > 0.0f ? lsum / cv : lsum;
+      } else {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int j0 = 64 * c + 2 * i;
+            const float p0 = ptx::ex2(x[j0] - m_run), p1 = ptx::ex2(x[j0 + 1] - m_run);
+            const float cv0 = colV[j0], cv1 = colV[j0 + 1];
+            r[i] = ptx::f32x2_to_f16x2(p0 * cv0, p1 * cv1);
+            const float t0 = __half2float(__ushort_as_half(static_cast<uint16_t>(r[i] & 0xFFFFu)));
+            const float t1 = __half2float(__ushort_as_half(static_cast<uint16_t>(r[i] >> 16)));
+            ls[i & 3] += (cv0 > 0.0f ? t0 / cv0 : p0) + (cv1 > 0.0f ? t1 / cv1 : p1);
+          }
+          ptx::tmem_st32(tS + 32 * c, r);
+        }
+        l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       }
-      l_run += lsum;
       ptx::tc_wait_st();
       ptx::tc_fence_before();
       __syncwarp();

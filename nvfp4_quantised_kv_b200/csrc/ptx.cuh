@@ -257,6 +257,17 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
   return r;
 }
 
+// acc + lo + hi of an f16x2 word, accumulated in fp32 (sm_100 mixed-precision add).
+__device__ __forceinline__ float add_f16x2_f32(float acc, uint32_t h2) {
+  asm("{\n\t.reg .f16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.f16 %0, lo, %0;\n\t"
+      "add.rn.f32.f16 %0, hi, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(h2));
+  return acc;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -36,9 +36,9 @@ def assert_cache_equal(cache, ocache, slots):
             a, b = got[:, :, s * Lc:(s + 1) * Lc], want[:, :, s * Lc:(s + 1) * Lc]
             bad = np.argwhere(a != b)
             assert bad.size == 0, f"{name} slot {s}: {len(bad)} bytes differ, first at {bad[:3].tolist()}"
-    for name in ("k_gscale", "v_gscale"):
+    for name, oname in (("k_gscale", "k_g"), ("v_gscale", "v_g")):
         got = getattr(cache, name).cpu().numpy()
-        want = getattr(ocache, name)
+        want = getattr(ocache, oname)
         for s in slots:
             assert np.array_equal(got[:, :, s].view(np.uint32), want[:, :, s].view(np.uint32)), name
 
