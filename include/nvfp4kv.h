@@ -106,6 +106,25 @@ int nvfp4_kv_quantize(const nvfp4kv_cache* cache, int32_t chunk_slot, const void
                       const void* v_bf16, int64_t token_stride, void* workspace,
                       size_t workspace_bytes, void* cuda_stream);
 
+/* nvfp4_kv_quantize without a workspace, for callers that cannot allocate device memory
+ * (a pre-planned arena sized before this library was linked, a host framework that owns
+ * every device allocation, a real-time loop that must not allocate).  The pages have no
+ * counterpart: this is a library convenience, not part of the method.
+ * Same arguments, results and errors as nvfp4_kv_quantize, except that the amax partials
+ * live in a fixed 64 KiB device array inside the library, which every GPU that loads the
+ * library keeps until the process exits.  It calls no cudaMalloc or cudaFree.
+ *  - Caches needing more partials than fit (2 * batch * heads * parts * 4 bytes, about
+ *    2 * batch * heads * 4 bytes for large batch * heads) are rejected with
+ *    NVFP4KV_ERR_WORKSPACE before anything is launched; use nvfp4_kv_quantize for them.
+ *  - The first call on each device looks up the array's device address (with that device
+ *    current), which may load the library's GPU code: make that first call before any
+ *    stream capture.
+ *  - All calls share the one array and every call overwrites what it reads, so nothing needs
+ *    clearing between calls; calls that may overlap on the GPU (unordered streams) race. */
+int nvfp4_kv_quantize_static_scratch(const nvfp4kv_cache* cache, int32_t chunk_slot,
+                                     const void* k_bf16, const void* v_bf16, int64_t token_stride,
+                                     void* cuda_stream);
+
 /* Attention of a chunk of bf16 queries over the NVFP4 cache.  The query chunk `q_chunk`
  * attends to the keys of the visible chunk slots
  *     V = { c < n_sink_chunks } U { q_chunk - window_chunks < c <= q_chunk },

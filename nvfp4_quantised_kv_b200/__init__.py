@@ -45,6 +45,7 @@ SIGNATURES = {
                                            ctypes.POINTER(_sz), ctypes.POINTER(_sz)]),
     "nvfp4kv_workspace_bytes": (_sz, [_CP, _i32]),
     "nvfp4_kv_quantize": (ctypes.c_int, [_CP, _i32, _vp, _vp, _i64, _vp, _sz, _vp]),
+    "nvfp4_kv_quantize_static_scratch": (ctypes.c_int, [_CP, _i32, _vp, _vp, _i64, _vp]),
     "nvfp4_kv_attention": (ctypes.c_int, [_CP, _vp, _i32, _i64, _i32, _i32, _i32, ctypes.c_float,
                                           _vp, _i32, _vp, _sz, _vp]),
     "nvfp4_kv_dequantize": (ctypes.c_int, [_CP, _i32, _i32, _i32, _vp, _vp]),

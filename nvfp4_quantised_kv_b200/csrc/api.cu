@@ -87,6 +87,28 @@ int nvfp4_kv_quantize(const nvfp4kv_cache* cache, int32_t chunk_slot, const void
   return e == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 
+int nvfp4_kv_quantize_static_scratch(const nvfp4kv_cache* cache, int32_t chunk_slot,
+                                     const void* k_bf16, const void* v_bf16, int64_t token_stride,
+                                     void* cuda_stream) {
+  int rc = check_cache(cache);
+  if (rc != NVFP4KV_OK) return rc;
+  if (chunk_slot < 0 || chunk_slot >= cache->capacity_chunks) return NVFP4KV_ERR_INVALID_ARG;
+  if (!k_bf16 || !v_bf16 || !aligned16(k_bf16) || !aligned16(v_bf16)) return NVFP4KV_ERR_INVALID_ARG;
+  if (token_stride < static_cast<int64_t>(cache->heads) * cache->head_dim || token_stride % 8 != 0)
+    return NVFP4KV_ERR_INVALID_ARG;
+  // The partials must fit the fixed array; larger caches have to use nvfp4_kv_quantize.
+  if (quantize_workspace_bytes(cache->batch, cache->heads, cache->chunk_tokens) > kStaticScratchBytes)
+    return NVFP4KV_ERR_WORKSPACE;
+  rc = check_device();
+  if (rc != NVFP4KV_OK) return rc;
+  void* scratch = nullptr;
+  if (static_scratch_address(&scratch) != cudaSuccess) return NVFP4KV_ERR_CUDA;
+  const cudaError_t e = launch_quantize(*cache, chunk_slot, static_cast<const uint16_t*>(k_bf16),
+                                        static_cast<const uint16_t*>(v_bf16), token_stride, scratch,
+                                        static_cast<cudaStream_t>(cuda_stream));
+  return e == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
+}
+
 int nvfp4_kv_attention(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q_tokens,
                        int64_t q_token_stride, int32_t q_chunk, int32_t n_sink_chunks,
                        int32_t window_chunks, float softmax_scale, void* out, int32_t out_dtype,

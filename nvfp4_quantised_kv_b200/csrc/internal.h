@@ -22,6 +22,10 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;
 // Number of amax partial slots per (b, h, tensor) and the workspace bytes they need.
 int quantize_parts(int batch, int heads, int chunk_tokens);
 size_t quantize_workspace_bytes(int batch, int heads, int chunk_tokens);
+// Size of the fixed device array the no-workspace quantiser variant uses for its partials.
+constexpr size_t kStaticScratchBytes = 64 * 1024;
+// Device address of that array on the current device (looked up on first use per device).
+cudaError_t static_scratch_address(void** out);
 cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
                             int64_t token_stride, void* workspace, cudaStream_t stream);
 

@@ -17,6 +17,8 @@
 // The second pass re-reads its input right after the first, from L2 for chunks that fit.
 // Every fp32 step uses an explicitly rounded intrinsic (no contraction, no flush to zero),
 // so the codes are bit-identical to the fp32 definition of the method.
+#include <mutex>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -197,4 +199,42 @@ cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k,
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------------------
+// Quantiser variant for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc or hand the library a workspace: code that runs
+// inside a pre-planned memory arena whose size was fixed before this library was linked,
+// plugins whose host framework owns every device allocation, and real-time loops where an
+// allocation could block or fragment the heap.  For them the amax partials live in this
+// file-scope array instead of a caller workspace.  Every GPU that loads the library keeps
+// the array (kStaticScratchBytes) until the process exits.  Each call overwrites all the
+// partials it reads, so nothing has to start at zero; all calls share the one array, so
+// calls that may overlap on the GPU (different streams without ordering) race on it.
+static __device__ __align__(256) uint32_t g_quant_scratch[kStaticScratchBytes / sizeof(uint32_t)];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+}  // namespace
+
+cudaError_t static_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    // Host code only holds a stand-in for the array's name; its device address has to be
+    // looked up once per device, with that device current.
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_quant_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
 }  // namespace nvfp4kv
+
