@@ -45,7 +45,7 @@ constexpr int BM = 128;  // query rows per tile (TMEM lanes)
 constexpr int BN = 128;  // keys per KV tile
 constexpr int D = kHeadDim;
 constexpr int NST = 2;   // stages of dequantised K / V tiles
-constexpr int NPK = 4;   // slots of packed data (K and V tiles alternate)
+constexpr int NPK = 3;   // slots of packed data (K and V tiles alternate)
 constexpr int PK_CODES = BN * kCodeBytes;               // 8192
 constexpr int PK_BYTES = PK_CODES + BN * kScaleBytes;   // 9216
 constexpr int TILE16 = BN * D * 2;                      // one 128 x 128 16-bit operand tile
@@ -66,12 +66,14 @@ struct Cfg {
   static constexpr int oK = oQ + QT * TILE16;
   static constexpr int oV = oK + NST * TILE16;
   static constexpr int oPK = oV + NST * TILE16;
-  static constexpr int oCol = oPK + NPK * PK_BYTES;  // per stage: colK[BN], colV[BN] (fp32)
+  static constexpr int oCol = oPK + NPK * PK_BYTES;      // per stage: colK[BN], colV[BN] (fp32)
   static constexpr int oInfo = oCol + NST * 2 * BN * 4;  // per stage: int4 {n_valid, uniform}
-  static constexpr int oBar = oInfo + NST * 16;
+  static constexpr int oRed = oInfo + NST * 16;          // per Q tile: 4 warp maxima
+  static constexpr int oBar = oRed + QT * 16;
   // barrier indices
   static constexpr int bQFull = 0;
-  static constexpr int bPkFull = 1;
+  static constexpr int bQReady = 1;
+  static constexpr int bPkFull = 2;
   static constexpr int bPkEmpty = bPkFull + NPK;
   static constexpr int bKFull = bPkEmpty + NPK;
   static constexpr int bVFull = bKFull + NST;
@@ -83,6 +85,7 @@ struct Cfg {
   static constexpr int kNumBars = bDrain + 1;
   static constexpr int oMisc = oBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag
   static constexpr int kSmemBytes = oMisc + 16 + 1024;  // + slack for 1024-B alignment
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 struct AttnParams {
@@ -113,7 +116,8 @@ __device__ __forceinline__ bool timed_out(uint64_t& t0, int& it) {
 }
 
 // Single-thread wait; gives up when another thread aborted or the limit is reached.
-__device__ __forceinline__ bool wait1(uint32_t bar, uint32_t parity, volatile uint32_t* abort, uint32_t* status) {
+__device__ __forceinline__ bool wait1(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
+                                      uint32_t* status) {
   uint64_t t0 = 0;
   int it = 0;
   while (!ptx::mbar_try_wait(bar, parity)) {
@@ -128,7 +132,8 @@ __device__ __forceinline__ bool wait1(uint32_t bar, uint32_t parity, volatile ui
 }
 
 // Warp-collective wait: every lane observes the phase; the give-up decision is uniform.
-__device__ __forceinline__ bool waitw(uint32_t bar, uint32_t parity, volatile uint32_t* abort, uint32_t* status) {
+__device__ __forceinline__ bool waitw(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
+                                      uint32_t* status) {
   const int lane = threadIdx.x & 31;
   uint64_t t0 = 0;
   int it = 0;
@@ -176,32 +181,36 @@ __device__ __forceinline__ float max_visible_gv(const AttnParams& p, int64_t bh)
   return m > 0.0f ? m : 1.0f;
 }
 
-// Dequantise one packed tile (codes + E4M3 scales of BN keys) into a 128B-swizzled
-// [key][d] operand tile of 16-bit values.  Thread dt of 128 handles 16 groups of 8
-// elements; a warp covers two keys (4 x 128 B rows) per step, conflict-free.
-template <bool kBF16>
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+  return __vmaxu2(a & 0x7FFF7FFFu, b & 0x7FFF7FFFu);
+}
+
+// Dequantise one packed tile (codes + E4M3 scales of BN keys) into a 128B-swizzled [key][d]
+// operand tile of fp16 values, code * scale (exact: <= 6 significant bits, 2^-10 .. 2688).
+// Thread dt of 128 handles one 16-element block per step (one scale conversion per block);
+// a warp covers four keys per step, its 16-byte stores spread evenly over the banks.
 __device__ __forceinline__ void dequant_tile(const uint8_t* pk, uint8_t* dst, int n, int dt) {
-#pragma unroll 4
-  for (int it = 0; it < 16; ++it) {
+#pragma unroll 2
+  for (int it = 0; it < 8; ++it) {
     const int job = it * 128 + dt;
-    const int key = job >> 4;
-    const int c16 = job & 15;
-    uint4 o = make_uint4(0, 0, 0, 0);
+    const int key = job >> 3;
+    const int blk = job & 7;
+    uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
     if (key < n) {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(pk + key * kCodeBytes + c16 * 4);
-      const uint32_t sb = pk[PK_CODES + key * kScaleBytes + (c16 >> 1)];
+      const uint2 w = *reinterpret_cast<const uint2*>(pk + key * kCodeBytes + blk * 8);
+      const uint32_t s2 = ptx::e4m3_to_f16x2_bcast(pk[PK_CODES + key * kScaleBytes + blk]);
       uint32_t h[4];
-      ptx::e2m1x8_to_f16x8(w, h);
-      const uint32_t s2 = ptx::e4m3_to_f16x2_bcast(sb);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        h[i] = ptx::hmul2_u32(h[i], s2);
-        if (kBF16) h[i] = ptx::f16x2_to_bf16x2(h[i]);
-      }
-      o = make_uint4(h[0], h[1], h[2], h[3]);
+      ptx::e2m1x8_to_f16x8(w.x, h);
+      o0 = make_uint4(ptx::hmul2_u32(h[0], s2), ptx::hmul2_u32(h[1], s2), ptx::hmul2_u32(h[2], s2),
+                      ptx::hmul2_u32(h[3], s2));
+      ptx::e2m1x8_to_f16x8(w.y, h);
+      o1 = make_uint4(ptx::hmul2_u32(h[0], s2), ptx::hmul2_u32(h[1], s2), ptx::hmul2_u32(h[2], s2),
+                      ptx::hmul2_u32(h[3], s2));
     }
-    const int off = (c16 >> 3) * HALF16 + key * 128 + (((c16 & 7) ^ (key & 7)) << 4);
-    *reinterpret_cast<uint4*>(dst + off) = o;
+    const int c0 = (blk * 2) & 7;  // 16-byte chunk of the 128-byte row (64 elements per half)
+    uint8_t* row = dst + (blk >> 2) * HALF16 + key * 128;
+    *reinterpret_cast<uint4*>(row + ((c0 ^ (key & 7)) << 4)) = o0;
+    *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ (key & 7)) << 4)) = o1;
   }
 }
 
@@ -225,6 +234,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar(C::bQFull), 1);
+    ptx::mbar_init(bar(C::bQReady), C::kSoftmaxWarps);
     for (int i = 0; i < NPK; ++i) {
       ptx::mbar_init(bar(C::bPkFull + i), 1);
       ptx::mbar_init(bar(C::bPkEmpty + i), C::kDequantWarps);
@@ -261,48 +271,93 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
     const uint32_t tS = tmem + lane_off + qt * BN;
     const uint32_t tO = tmem + lane_off + QT * BN + qt * D;
     const float gv_ref = max_visible_gv(p, bh);
+    bool ok = waitw(bar(C::bQFull), 0, abort_flag, p.status);
+    float pre_scale = 1.0f;
+
+    // ---- Q tile: bf16 -> fp16 in place, exact, after a power-of-two prescale 2^-e that keeps
+    // the tile's largest |q| below 2^15; S is scaled back by 2^e with the logit factor.
+    float q_unscale = 1.0f;
+    uint8_t* qrow = smem + C::oQ + qt * TILE16 + row * 128;
+    {
+      uint32_t mb = 0;
+      if (ok) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint4 v = *reinterpret_cast<const uint4*>(qrow + (i >> 3) * HALF16 + (((i + lane) & 7) << 4));
+          mb = __vmaxu2(mb, __vmaxu2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w)));
+        }
+      }
+      mb = max(mb & 0xFFFFu, mb >> 16);
+      mb = __reduce_max_sync(0xFFFFFFFFu, mb);
+      uint32_t* red = reinterpret_cast<uint32_t*>(smem + C::oRed + qt * 16);
+      if (lane == 0) red[warp & 3] = mb;
+      ptx::named_bar(1 + qt, 128);  // reached by all four warps of the tile, on every path
+      mb = max(max(red[0], red[1]), max(red[2], red[3]));
+      const int ex = static_cast<int>((mb >> 7) & 0xFF) - 127;  // floor(log2 max|q|)
+      const int e = ex > 14 ? ex - 14 : 0;
+      q_unscale = __int_as_float((127 + e) << 23);  // 2^e
+      pre_scale = __int_as_float((127 - e) << 23);  // 2^-e
+    }
+    if (ok) {
+#pragma unroll 4
+      for (int i = 0; i < 16; ++i) {
+        uint4* ptr = reinterpret_cast<uint4*>(qrow + (i >> 3) * HALF16 + (((i + lane) & 7) << 4));
+        const uint4 v = *ptr;
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          o[k] = ptx::f32x2_to_f16x2(__uint_as_float(wv[k] << 16) * pre_scale,
+                                     __uint_as_float(wv[k] & 0xFFFF0000u) * pre_scale);
+        *ptr = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(C::bQReady));
+    }
+
     float m_run = -INFINITY, l_run = 0.0f;
-    bool ok = true;
     for (int j = 0; j < p.n_tiles && ok; ++j) {
       const int st = j % NST;
       ok = waitw(bar(C::bSFull + qt), j & 1, abort_flag, p.status) &&
            waitw(bar(C::bKFull + st), (j / NST) & 1, abort_flag, p.status);
       if (!ok) break;
       ptx::tc_fence_after();
-      float x[BN];
-      {
-        uint32_t r[32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          ptx::tmem_ld32(tS + 32 * c, r);
-          ptx::tc_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(r[i]);
-        }
-      }
       const int4 info = *reinterpret_cast<const int4*>(smem + C::oInfo + 16 * st);
       const float* colK = reinterpret_cast<const float*>(smem + C::oCol + st * 2 * BN * 4);
       const float* colV = colK + BN;
-      // Row maximum of the log2-domain logits x = S * g_K(chunk) * scale * log2(e).  In a
-      // tile inside one chunk (info.y) x stays unscaled here: g_K >= 0 scales the maximum.
+      const float ck = colK[0] * q_unscale;
+
+      // ---- pass 1: row maximum of x = S * g_K(chunk) * scale * log2(e)
       float mx;
-      if (info.y) {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      {
+        float ma = -INFINITY, mb = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < BN; ++i) m4[i & 3] = fmaxf(m4[i & 3], x[i]);
-        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * colK[0];
-      } else {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tS + 32 * c, r);
+          ptx::tc_wait_ld();
+          if (info.y) {
 #pragma unroll
-        for (int i = 0; i < BN; ++i) {
-          x[i] = (i < info.x) ? x[i] * colK[i] : -INFINITY;
-          m4[i & 3] = fmaxf(m4[i & 3], x[i]);
+            for (int i = 0; i < 32; i += 4) {
+              ma = ptx::fmax3(ma, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+              mb = ptx::fmax3(mb, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int jj = 32 * c + i;
+              const float xv = jj < info.x ? __uint_as_float(r[i]) * colK[jj] * q_unscale : -INFINITY;
+              ma = fmaxf(ma, xv);
+            }
+          }
         }
-        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        mx = info.y ? fmaxf(ma, mb) * ck : fmaxf(ma, mb);
       }
-      // Lazy rescale: a row moves its running max only when it grew by more than 2^8.  The
-      // O rescale uses warp-collective TMEM accesses, so it runs for the whole warp when any
-      // row of the warp moved (alpha = 1 for the rows that did not).
+
+      // ---- lazy rescale: a row moves its running max only when it grew by more than 2^8.  The
+      // O rescale uses warp-collective TMEM accesses, so it runs for the whole warp when any row
+      // of the warp moved (alpha = 1 for the rows that did not).
       const bool moved = mx > m_run + 8.0f;
       float alpha = 1.0f;
       if (moved) {
@@ -324,50 +379,62 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
           ptx::tmem_st32(tO + 32 * c, r);
         }
       }
-      // P~ = 2^(x - m) * cv, cv = g_V(chunk) / max g_V, rounded to fp16 pairs and written over
-      // S's first 64 TMEM columns (S is fully in registers by now).  The row sum l adds the
-      // same rounded values divided by cv, so the rounding of P~ largely cancels in O / l.
-      // A key of an all-zero V chunk (cv = 0) contributes 0 to O and its p to l.
-      float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+
+      // ---- pass 2: P~ = 2^(x - m) * cv with cv = g_V(chunk) / max g_V, rounded to fp16 pairs and
+      // written over the S columns already read (chunk c -> P columns [16c, 16c + 16)).  The row
+      // sum adds the same rounded values divided by cv, so the rounding of P~ largely cancels in
+      // O / l; a key of an all-zero V chunk (cv = 0) adds 0 to O and its p to l.
+      float la = 0.0f, lb = 0.0f;
       if (info.y) {
-        const float ck = colK[0], cv = colV[0];
+        const float cv = colV[0];
         const float mneg = (cv > 0.0f ? log2f(cv) : 0.0f) - m_run;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t r[32];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32], pk[16];
+          ptx::tmem_ld32(tS + 32 * c, r);
+          ptx::tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float p0 = ptx::ex2(fmaf(x[64 * c + 2 * i], ck, mneg));
-            const float p1 = ptx::ex2(fmaf(x[64 * c + 2 * i + 1], ck, mneg));
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ptx::ex2(fmaf(__uint_as_float(r[2 * i]), ck, mneg));
+            const float p1 = ptx::ex2(fmaf(__uint_as_float(r[2 * i + 1]), ck, mneg));
             if (cv > 0.0f) {
-              r[i] = ptx::f32x2_to_f16x2(p0, p1);
-              ls[i & 3] = ptx::add_f16x2_f32(ls[i & 3], r[i]);
+              pk[i] = ptx::f32x2_to_f16x2(p0, p1);
+              if (i & 1)
+                lb = ptx::add_f16x2_f32(lb, pk[i]);
+              else
+                la = ptx::add_f16x2_f32(la, pk[i]);
             } else {
-              r[i] = 0u;
-              ls[i & 3] += p0 + p1;
+              pk[i] = 0u;
+              la += p0;
+              lb += p1;
             }
           }
-          ptx::tmem_st32(tS + 32 * c, r);
+          ptx::tmem_st16(tS + 16 * c, pk);
         }
-        const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
-        l_run += cv > 0.0f ? lsum / cv : lsum;
+        l_run += cv > 0.0f ? (la + lb) / cv : la + lb;
       } else {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32], pk[16];
+          ptx::tmem_ld32(tS + 32 * c, r);
+          ptx::tc_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t r[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int j0 = 64 * c + 2 * i;
-            const float p0 = ptx::ex2(x[j0] - m_run), p1 = ptx::ex2(x[j0 + 1] - m_run);
+          for (int i = 0; i < 16; ++i) {
+            const int j0 = 32 * c + 2 * i;
+            const float x0 = j0 < info.x ? __uint_as_float(r[2 * i]) * colK[j0] * q_unscale : -INFINITY;
+            const float x1 =
+                j0 + 1 < info.x ? __uint_as_float(r[2 * i + 1]) * colK[j0 + 1] * q_unscale : -INFINITY;
+            const float p0 = ptx::ex2(x0 - m_run), p1 = ptx::ex2(x1 - m_run);
             const float cv0 = colV[j0], cv1 = colV[j0 + 1];
-            r[i] = ptx::f32x2_to_f16x2(p0 * cv0, p1 * cv1);
-            const float t0 = __half2float(__ushort_as_half(static_cast<uint16_t>(r[i] & 0xFFFFu)));
-            const float t1 = __half2float(__ushort_as_half(static_cast<uint16_t>(r[i] >> 16)));
-            ls[i & 3] += (cv0 > 0.0f ? t0 / cv0 : p0) + (cv1 > 0.0f ? t1 / cv1 : p1);
+            pk[i] = ptx::f32x2_to_f16x2(p0 * cv0, p1 * cv1);
+            const float t0 = __half2float(__ushort_as_half(static_cast<uint16_t>(pk[i] & 0xFFFFu)));
+            const float t1 = __half2float(__ushort_as_half(static_cast<uint16_t>(pk[i] >> 16)));
+            la += cv0 > 0.0f ? t0 / cv0 : p0;
+            lb += cv1 > 0.0f ? t1 / cv1 : p1;
           }
-          ptx::tmem_st32(tS + 32 * c, r);
+          ptx::tmem_st16(tS + 16 * c, pk);
         }
-        l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        l_run += la + lb;
       }
       ptx::tc_wait_st();
       ptx::tc_fence_before();
@@ -454,30 +521,35 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
   } else if (warp == C::kMmaWarp) {
     // ============================================================ MMA issuer
     if (lane == 0) {
-      // kind::f16 instruction descriptors: fp32 accumulate; M = 128; N = 128.
-      constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) |  // bf16 x bf16, both K-major
+      // kind::f16 instruction descriptors: fp16 x fp16 -> fp32; M = 128; N = 128.
+      constexpr uint32_t kIdescQK = (1u << 4) |  // A = Q and B = K^ both K-major
                                     (static_cast<uint32_t>(BN >> 3) << 17) |
                                     (static_cast<uint32_t>(BM >> 4) << 24);
-      constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) |  // fp16 x fp16, B (V) MN-major
+      constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) |  // B = V^ MN-major
                                     (static_cast<uint32_t>(D >> 3) << 17) |
                                     (static_cast<uint32_t>(BM >> 4) << 24);
-      bool ok = wait1(bar(C::bQFull), 0, abort_flag, p.status);
+      auto issue_qk = [&](int q, int st) {
+        const uint32_t sQ = sbase + C::oQ + q * TILE16;
+        const uint32_t sK = sbase + C::oK + st * TILE16;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * HALF16 + (kk & 3) * 32;
+          ptx::mma_ss(tmem + q * BN, ptx::smem_desc_sw128(sQ + koff, 16, 1024),
+                      ptx::smem_desc_sw128(sK + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(bar(C::bSFull + q));
+      };
+      bool ok = wait1(bar(C::bQReady), 0, abort_flag, p.status) && p.n_tiles > 0 &&
+                wait1(bar(C::bKFull + 0), 0, abort_flag, p.status);
+      if (ok) {
+        ptx::tc_fence_after();
+        for (int q = 0; q < QT; ++q) issue_qk(q, 0);
+      }
+      // Per KV tile j: PV(q, j) as soon as softmax q has written P(q, j), then QK(q, j + 1) into
+      // the same S columns; the two query tiles alternate so the tensor core always has the
+      // other tile's work while one softmax runs.
       for (int j = 0; j < p.n_tiles && ok; ++j) {
         const int st = j % NST;
-        ok = wait1(bar(C::bKFull + st), (j / NST) & 1, abort_flag, p.status);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        const uint32_t sK = sbase + C::oK + st * TILE16;
-        for (int q = 0; q < QT; ++q) {
-          const uint32_t sQ = sbase + C::oQ + q * TILE16;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * HALF16 + (kk & 3) * 32;
-            ptx::mma_ss(tmem + q * BN, ptx::smem_desc_sw128(sQ + koff, 16, 1024),
-                        ptx::smem_desc_sw128(sK + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
-          }
-          ptx::mma_commit(bar(C::bSFull + q));
-        }
         const uint32_t sV = sbase + C::oV + st * TILE16;
         for (int q = 0; q < QT && ok; ++q) {
           ok = wait1(bar(C::bPFull + q), j & 1, abort_flag, p.status);
@@ -490,8 +562,17 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
                         ptx::smem_desc_sw128(sV + kk * 2048, HALF16, 1024), kIdescPV,
                         (j > 0 || kk > 0) ? 1u : 0u);
           ptx::mma_commit(bar(C::bODone + q));
+          if (q == QT - 1) ptx::mma_commit(bar(C::bKvEmpty + st));
+          if (j + 1 < p.n_tiles) {
+            const int st1 = (j + 1) % NST;
+            if (q == 0) {
+              ok = wait1(bar(C::bKFull + st1), ((j + 1) / NST) & 1, abort_flag, p.status);
+              if (!ok) break;
+              ptx::tc_fence_after();
+            }
+            issue_qk(q, st1);
+          }
         }
-        if (ok) ptx::mma_commit(bar(C::bKvEmpty + st));
       }
       // every MMA issued so far completes before the drain barrier's phase 0
       ptx::mma_commit(bar(C::bDrain));
@@ -515,8 +596,8 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
         ok = waitw(bar(C::bPkFull + slot), (pk / NPK) & 1, abort_flag, p.status);
         if (!ok) break;
         const uint8_t* src = smem + C::oPK + slot * PK_BYTES;
+        dequant_tile(src, smem + (t == 0 ? C::oK : C::oV) + st * TILE16, n, dt);
         if (t == 0) {
-          dequant_tile<true>(src, smem + C::oK + st * TILE16, n, dt);
           float* colK = reinterpret_cast<float*>(smem + C::oCol + st * 2 * BN * 4);
           const bool valid = dt < n;
           const int c = valid ? (key0 + dt) / p.Lc : 0;
@@ -526,8 +607,6 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
             const int uniform = (n == BN) && (key0 / p.Lc == (key0 + BN - 1) / p.Lc);
             *reinterpret_cast<int4*>(smem + C::oInfo + 16 * st) = make_int4(n, uniform, 0, 0);
           }
-        } else {
-          dequant_tile<false>(src, smem + C::oV + st * TILE16, n, dt);
         }
         ptx::fence_proxy_async_smem();
         __syncwarp();
@@ -635,7 +714,7 @@ int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, in
                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return NVFP4KV_ERR_CUDA;
-  const cudaError_t e = launch<1>(tm, prm, stream);
+  const cudaError_t e = q_tokens <= BM ? launch<1>(tm, prm, stream) : launch<2>(tm, prm, stream);
   return e == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 

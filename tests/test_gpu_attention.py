@@ -120,3 +120,22 @@ def test_query_token_stride_and_softmax_scale():
                          for i in range(w.q_tokens)], np.int32)
         want = oracle.attention_rows(qb, ocache, w.q_chunk, w.n_sink, w.window, rows, scale)
         assert_attention_close(gather_rows(out.cpu().numpy(), rows), want, f"scale {scale}")
+
+
+def test_queries_beyond_fp16_range_use_an_exact_power_of_two_prescale():
+    # |q| up to ~2^22 (beyond fp16) with K scaled down by the same factor: logits stay moderate
+    from tests._bf16 import bf16_bits_to_f32, f32_to_bf16_bits
+    w = dataclasses.replace(W["tiny"], **EDGE["ragged_two_runs"])
+    cache, ocache = make_caches(w, [])
+    for slot in w.visible_chunks:
+        k, v = synthetic.chunk_kv(w, slot)
+        k = f32_to_bf16_bits(bf16_bits_to_f32(k) * np.float32(2.0 ** -20))
+        cache.quantize(slot, dev_bf16(k), dev_bf16(v))
+        ocache.append(slot, k, v)
+    qb = f32_to_bf16_bits(bf16_bits_to_f32(synthetic.queries(w)) * np.float32(2.0 ** 20))
+    out = cache.attention(dev_bf16(qb), w.q_chunk, w.n_sink, w.window)
+    assert cache.read_status() == 0
+    rows = np.array([(b, h, i) for b in range(w.batch) for h in range(w.heads)
+                     for i in range(w.q_tokens)], np.int32)
+    want = oracle.attention_rows(qb, ocache, w.q_chunk, w.n_sink, w.window, rows)
+    assert_attention_close(gather_rows(out.cpu().numpy(), rows), want, "large q")
