@@ -187,30 +187,45 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
 
 // Dequantise one packed tile (codes + E4M3 scales of BN keys) into a 128B-swizzled [key][d]
 // operand tile of fp16 values, code * scale (exact: <= 6 significant bits, 2^-10 .. 2688).
-// Thread dt of 128 handles one 16-element block per step (one scale conversion per block);
-// a warp covers four keys per step, its 16-byte stores spread evenly over the banks.
+// Thread dt of 128 handles eight 16-element blocks (one scale conversion per block), four at a
+// time with all their shared-memory loads issued first; a warp covers four keys per block step.
 __device__ __forceinline__ void dequant_tile(const uint8_t* pk, uint8_t* dst, int n, int dt) {
-#pragma unroll 2
-  for (int it = 0; it < 8; ++it) {
-    const int job = it * 128 + dt;
-    const int key = job >> 3;
-    const int blk = job & 7;
-    uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
-    if (key < n) {
-      const uint2 w = *reinterpret_cast<const uint2*>(pk + key * kCodeBytes + blk * 8);
-      const uint32_t s2 = ptx::e4m3_to_f16x2_bcast(pk[PK_CODES + key * kScaleBytes + blk]);
-      uint32_t h[4];
-      ptx::e2m1x8_to_f16x8(w.x, h);
-      o0 = make_uint4(ptx::hmul2_u32(h[0], s2), ptx::hmul2_u32(h[1], s2), ptx::hmul2_u32(h[2], s2),
-                      ptx::hmul2_u32(h[3], s2));
-      ptx::e2m1x8_to_f16x8(w.y, h);
-      o1 = make_uint4(ptx::hmul2_u32(h[0], s2), ptx::hmul2_u32(h[1], s2), ptx::hmul2_u32(h[2], s2),
-                      ptx::hmul2_u32(h[3], s2));
+#pragma unroll 1
+  for (int base = 0; base < 8; base += 4) {
+    uint2 w[4];
+    uint32_t sb[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int job = (base + u) * 128 + dt;
+      const int key = job >> 3, blk = job & 7;
+      w[u] = *reinterpret_cast<const uint2*>(pk + key * kCodeBytes + blk * 8);
+      sb[u] = pk[PK_CODES + key * kScaleBytes + blk];
     }
-    const int c0 = (blk * 2) & 7;  // 16-byte chunk of the 128-byte row (64 elements per half)
-    uint8_t* row = dst + (blk >> 2) * HALF16 + key * 128;
-    *reinterpret_cast<uint4*>(row + ((c0 ^ (key & 7)) << 4)) = o0;
-    *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ (key & 7)) << 4)) = o1;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int job = (base + u) * 128 + dt;
+      const int key = job >> 3, blk = job & 7;
+      const uint32_t s2 = ptx::e4m3_to_f16x2_bcast(sb[u]);
+      uint32_t h[4], g[4];
+      ptx::e2m1x8_to_f16x8(w[u].x, h);
+      ptx::e2m1x8_to_f16x8(w[u].y, g);
+      uint4 o0 = make_uint4(ptx::hmul2_u32(h[0], s2), ptx::hmul2_u32(h[1], s2), ptx::hmul2_u32(h[2], s2),
+                            ptx::hmul2_u32(h[3], s2));
+      uint4 o1 = make_uint4(ptx::hmul2_u32(g[0], s2), ptx::hmul2_u32(g[1], s2), ptx::hmul2_u32(g[2], s2),
+                            ptx::hmul2_u32(g[3], s2));
+      if (key >= n) {  // past the run's last key: zero rows (P is 0 there, 0 * 0 stays 0)
+        o0 = make_uint4(0, 0, 0, 0);
+        o1 = o0;
+      }
+      // 16-byte chunks c0, c0 + 1 of the 128-byte row (64 elements per half).  A 16-byte warp
+      // store is served in phases of 8 lanes (one key, both halves of the row); lanes of the
+      // second half store their odd chunk first, so the 8 lanes of a phase hit 8 distinct banks.
+      const int c0 = (blk * 2) & 7;
+      const bool swap = blk >= 4;
+      uint8_t* row = dst + (blk >> 2) * HALF16 + key * 128;
+      *reinterpret_cast<uint4*>(row + (((c0 + (swap ? 1 : 0)) ^ (key & 7)) << 4)) = swap ? o1 : o0;
+      *reinterpret_cast<uint4*>(row + (((c0 + (swap ? 0 : 1)) ^ (key & 7)) << 4)) = swap ? o0 : o1;
+    }
   }
 }
 
@@ -328,114 +343,138 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       const float* colV = colK + BN;
       const float ck = colK[0] * q_unscale;
 
-      // ---- pass 1: row maximum of x = S * g_K(chunk) * scale * log2(e)
-      float mx;
-      {
-        float ma = -INFINITY, mb = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          ptx::tmem_ld32(tS + 32 * c, r);
-          ptx::tc_wait_ld();
-          if (info.y) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              ma = ptx::fmax3(ma, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-              mb = ptx::fmax3(mb, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int jj = 32 * c + i;
-              const float xv = jj < info.x ? __uint_as_float(r[i]) * colK[jj] * q_unscale : -INFINITY;
-              ma = fmaxf(ma, xv);
-            }
-          }
-        }
-        mx = info.y ? fmaxf(ma, mb) * ck : fmaxf(ma, mb);
-      }
-
-      // ---- lazy rescale: a row moves its running max only when it grew by more than 2^8.  The
-      // O rescale uses warp-collective TMEM accesses, so it runs for the whole warp when any row
-      // of the warp moved (alpha = 1 for the rows that did not).
-      const bool moved = mx > m_run + 8.0f;
-      float alpha = 1.0f;
-      if (moved) {
-        alpha = ptx::ex2(m_run - mx);
-        l_run *= alpha;
-        m_run = mx;
-      }
-      if (j > 0 && __any_sync(0xFFFFFFFFu, moved)) {
-        ok = waitw(bar(C::bODone + qt), (j - 1) & 1, abort_flag, p.status);
-        if (!ok) break;
-        ptx::tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          ptx::tmem_ld32(tO + 32 * c, r);
-          ptx::tc_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          ptx::tmem_st32(tO + 32 * c, r);
-        }
-      }
-
-      // ---- pass 2: P~ = 2^(x - m) * cv with cv = g_V(chunk) / max g_V, rounded to fp16 pairs and
-      // written over the S columns already read (chunk c -> P columns [16c, 16c + 16)).  The row
-      // sum adds the same rounded values divided by cv, so the rounding of P~ largely cancels in
-      // O / l; a key of an all-zero V chunk (cv = 0) adds 0 to O and its p to l.
-      float la = 0.0f, lb = 0.0f;
-      if (info.y) {
+      // P~ = 2^(x - m) * cv with cv = g_V(chunk) / max g_V, rounded to fp16 pairs (64 registers),
+      // then written over S's first 64 TMEM columns.  The row sum adds the same rounded values
+      // divided by cv, so the rounding of P~ largely cancels in O / l.
+      uint32_t pk[64];
+      bool redo = true;
+      if (j > 0 && info.y && colV[0] > 0.0f) {
+        // Common case, one pass: exponentiate against the running max while tracking the tile
+        // maximum; valid unless some row's maximum grew by more than 2^8.
         const float cv = colV[0];
-        const float mneg = (cv > 0.0f ? log2f(cv) : 0.0f) - m_run;
+        const float mneg = log2f(cv) - m_run;
+        float ma = -INFINITY, mb = -INFINITY, la = 0.0f, lb = 0.0f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t r[32], pk[16];
+          uint32_t r[32];
           ptx::tmem_ld32(tS + 32 * c, r);
           ptx::tc_wait_ld();
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = ptx::ex2(fmaf(__uint_as_float(r[2 * i]), ck, mneg));
-            const float p1 = ptx::ex2(fmaf(__uint_as_float(r[2 * i + 1]), ck, mneg));
-            if (cv > 0.0f) {
-              pk[i] = ptx::f32x2_to_f16x2(p0, p1);
-              if (i & 1)
-                lb = ptx::add_f16x2_f32(lb, pk[i]);
-              else
-                la = ptx::add_f16x2_f32(la, pk[i]);
+            const float s0 = __uint_as_float(r[2 * i]), s1 = __uint_as_float(r[2 * i + 1]);
+            if (i & 1) mb = ptx::fmax3(mb, s0, s1); else ma = ptx::fmax3(ma, s0, s1);
+            pk[16 * c + i] = ptx::f32x2_to_f16x2(ptx::ex2(fmaf(s0, ck, mneg)), ptx::ex2(fmaf(s1, ck, mneg)));
+            if (i & 1) lb = ptx::add_f16x2_f32(lb, pk[16 * c + i]);
+            else la = ptx::add_f16x2_f32(la, pk[16 * c + i]);
+          }
+        }
+        redo = __any_sync(0xFFFFFFFFu, fmaxf(ma, mb) * ck > m_run + 8.0f);
+        if (!redo) l_run += (la + lb) / cv;
+      }
+      if (redo) {
+        // General case (first tile, a tile across chunk boundaries or with masked keys, an
+        // all-zero V chunk, or a jump of the maximum): exact row maximum first.
+        float mx;
+        {
+          float ma = -INFINITY, mb = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(tS + 32 * c, r);
+            ptx::tc_wait_ld();
+            if (info.y) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) {
+                ma = ptx::fmax3(ma, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+                mb = ptx::fmax3(mb, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+              }
             } else {
-              pk[i] = 0u;
-              la += p0;
-              lb += p1;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int jj = 32 * c + i;
+                ma = fmaxf(ma, jj < info.x ? __uint_as_float(r[i]) * colK[jj] * q_unscale : -INFINITY);
+              }
             }
           }
-          ptx::tmem_st16(tS + 16 * c, pk);
+          mx = info.y ? fmaxf(ma, mb) * ck : fmaxf(ma, mb);
         }
-        l_run += cv > 0.0f ? (la + lb) / cv : la + lb;
-      } else {
+        // Lazy rescale: a row moves its running max only when it grew by more than 2^8.  The O
+        // rescale uses warp-collective TMEM accesses, so it runs for the whole warp when any
+        // row of the warp moved (alpha = 1 for the rows that did not).
+        const bool moved = mx > m_run + 8.0f;
+        float alpha = 1.0f;
+        if (moved) {
+          alpha = ptx::ex2(m_run - mx);
+          l_run *= alpha;
+          m_run = mx;
+        }
+        if (j > 0 && __any_sync(0xFFFFFFFFu, moved)) {
+          ok = waitw(bar(C::bODone + qt), (j - 1) & 1, abort_flag, p.status);
+          if (!ok) break;
+          ptx::tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32], pk[16];
-          ptx::tmem_ld32(tS + 32 * c, r);
-          ptx::tc_wait_ld();
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(tO + 32 * c, r);
+            ptx::tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int j0 = 32 * c + 2 * i;
-            const float x0 = j0 < info.x ? __uint_as_float(r[2 * i]) * colK[j0] * q_unscale : -INFINITY;
-            const float x1 =
-                j0 + 1 < info.x ? __uint_as_float(r[2 * i + 1]) * colK[j0 + 1] * q_unscale : -INFINITY;
-            const float p0 = ptx::ex2(x0 - m_run), p1 = ptx::ex2(x1 - m_run);
-            const float cv0 = colV[j0], cv1 = colV[j0 + 1];
-            pk[i] = ptx::f32x2_to_f16x2(p0 * cv0, p1 * cv1);
-            const float t0 = __half2float(__ushort_as_half(static_cast<uint16_t>(pk[i] & 0xFFFFu)));
-            const float t1 = __half2float(__ushort_as_half(static_cast<uint16_t>(pk[i] >> 16)));
-            la += cv0 > 0.0f ? t0 / cv0 : p0;
-            lb += cv1 > 0.0f ? t1 / cv1 : p1;
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            ptx::tmem_st32(tO + 32 * c, r);
           }
-          ptx::tmem_st16(tS + 16 * c, pk);
         }
-        l_run += la + lb;
+        float la = 0.0f, lb = 0.0f;
+        if (info.y) {
+          // a key of an all-zero V chunk (cv = 0) adds 0 to O and its p to l
+          const float cv = colV[0];
+          const float mneg = (cv > 0.0f ? log2f(cv) : 0.0f) - m_run;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(tS + 32 * c, r);
+            ptx::tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float p0 = ptx::ex2(fmaf(__uint_as_float(r[2 * i]), ck, mneg));
+              const float p1 = ptx::ex2(fmaf(__uint_as_float(r[2 * i + 1]), ck, mneg));
+              if (cv > 0.0f) {
+                pk[16 * c + i] = ptx::f32x2_to_f16x2(p0, p1);
+                if (i & 1) lb = ptx::add_f16x2_f32(lb, pk[16 * c + i]);
+                else la = ptx::add_f16x2_f32(la, pk[16 * c + i]);
+              } else {
+                pk[16 * c + i] = 0u;
+                la += p0;
+                lb += p1;
+              }
+            }
+          }
+          l_run += cv > 0.0f ? (la + lb) / cv : la + lb;
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(tS + 32 * c, r);
+            ptx::tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int j0 = 32 * c + 2 * i;
+              const float x0 = j0 < info.x ? __uint_as_float(r[2 * i]) * colK[j0] * q_unscale : -INFINITY;
+              const float x1 =
+                  j0 + 1 < info.x ? __uint_as_float(r[2 * i + 1]) * colK[j0 + 1] * q_unscale : -INFINITY;
+              const float p0 = ptx::ex2(x0 - m_run), p1 = ptx::ex2(x1 - m_run);
+              const float cv0 = colV[j0], cv1 = colV[j0 + 1];
+              const uint32_t w = ptx::f32x2_to_f16x2(p0 * cv0, p1 * cv1);
+              pk[16 * c + i] = w;
+              const float t0 = __half2float(__ushort_as_half(static_cast<uint16_t>(w & 0xFFFFu)));
+              const float t1 = __half2float(__ushort_as_half(static_cast<uint16_t>(w >> 16)));
+              la += cv0 > 0.0f ? t0 / cv0 : p0;
+              lb += cv1 > 0.0f ? t1 / cv1 : p1;
+            }
+          }
+          l_run += la + lb;
+        }
       }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) ptx::tmem_st16p(tS + 16 * c, &pk[16 * c]);
       ptx::tc_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
