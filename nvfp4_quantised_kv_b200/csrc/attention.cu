@@ -58,8 +58,9 @@ struct Cfg {
   static constexpr int kProducerWarp = kSoftmaxWarps;
   static constexpr int kMmaWarp = kSoftmaxWarps + 1;
   static constexpr int kDequantWarp0 = kSoftmaxWarps + 2;
-  static constexpr int kDequantWarps = 4;
-  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2 + kDequantWarps);
+  static constexpr int kDequantWarps = 6;  // 2 in the producer/MMA warpgroup + one full warpgroup
+  static constexpr int kDequantThreads = 32 * kDequantWarps;
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2 + kDequantWarps);  // whole warpgroups
   static constexpr uint32_t kTmemCols = QT == 1 ? 256 : 512;
   // shared memory map (bytes from a 1024-aligned base)
   static constexpr int oQ = 0;
@@ -187,23 +188,28 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
 
 // Dequantise one packed tile (codes + E4M3 scales of BN keys) into a 128B-swizzled [key][d]
 // operand tile of fp16 values, code * scale (exact: <= 6 significant bits, 2^-10 .. 2688).
-// Thread dt of 128 handles eight 16-element blocks (one scale conversion per block), four at a
-// time with all their shared-memory loads issued first; a warp covers four keys per block step.
+// The 1024 16-element blocks of a tile are dealt round-robin to NT threads, three at a time
+// with all their shared-memory loads issued first (one scale conversion per block).
+template <int NT>
 __device__ __forceinline__ void dequant_tile(const uint8_t* pk, uint8_t* dst, int n, int dt) {
+  constexpr int kPer = (1024 + NT - 1) / NT;  // blocks per thread, rounded up
 #pragma unroll 1
-  for (int base = 0; base < 8; base += 4) {
-    uint2 w[4];
-    uint32_t sb[4];
+  for (int base = 0; base < kPer; base += 3) {
+    uint2 w[3];
+    uint32_t sb[3];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int job = (base + u) * 128 + dt;
-      const int key = job >> 3, blk = job & 7;
-      w[u] = *reinterpret_cast<const uint2*>(pk + key * kCodeBytes + blk * 8);
-      sb[u] = pk[PK_CODES + key * kScaleBytes + blk];
+    for (int u = 0; u < 3; ++u) {
+      const int job = (base + u) * NT + dt;
+      if (base + u < kPer && job < 1024) {
+        const int key = job >> 3, blk = job & 7;
+        w[u] = *reinterpret_cast<const uint2*>(pk + key * kCodeBytes + blk * 8);
+        sb[u] = pk[PK_CODES + key * kScaleBytes + blk];
+      }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int job = (base + u) * 128 + dt;
+    for (int u = 0; u < 3; ++u) {
+      const int job = (base + u) * NT + dt;
+      if (base + u >= kPer || job >= 1024) continue;
       const int key = job >> 3, blk = job & 7;
       const uint32_t s2 = ptx::e4m3_to_f16x2_bcast(sb[u]);
       uint32_t h[4], g[4];
@@ -277,9 +283,15 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = misc[0];
+  // Registers move from the producer/MMA/dequant warpgroups (80 each) to the two softmax
+  // warpgroups (176 each), which hold a whole 128-column S row: 2*128*176 + 2*128*80 = 65536,
+  // exactly what the 512-thread block was launched with.  Each role branch starts with its
+  // warpgroup's budget change.
+  static_assert(QT == 1 || C::kThreads == 512, "register split assumes four warpgroups");
 
   if (warp < C::kSoftmaxWarps) {
     // ============================================================ softmax + epilogue
+    if constexpr (QT == 2) ptx::setmaxnreg_inc<176>();
     const int qt = warp >> 2;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -342,139 +354,108 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       const float* colK = reinterpret_cast<const float*>(smem + C::oCol + st * 2 * BN * 4);
       const float* colV = colK + BN;
       const float ck = colK[0] * q_unscale;
+      // A tile inside one chunk with every key valid and a nonzero V scale takes the uniform path
+      // (one logit factor, one cv); any other tile works per column.
+      const bool uni = info.y && colV[0] > 0.0f;
 
-      // P~ = 2^(x - m) * cv with cv = g_V(chunk) / max g_V, rounded to fp16 pairs (64 registers),
-      // then written over S's first 64 TMEM columns.  The row sum adds the same rounded values
-      // divided by cv, so the rounding of P~ largely cancels in O / l.
-      uint32_t pk[64];
-      bool redo = true;
-      if (j > 0 && info.y && colV[0] > 0.0f) {
-        // Common case, one pass: exponentiate against the running max while tracking the tile
-        // maximum; valid unless some row's maximum grew by more than 2^8.
-        const float cv = colV[0];
-        const float mneg = log2f(cv) - m_run;
-        float ma = -INFINITY, mb = -INFINITY, la = 0.0f, lb = 0.0f;
+      // The whole 128-column S row: four loads in flight, one wait.
+      uint32_t sr[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          ptx::tmem_ld32(tS + 32 * c, r);
-          ptx::tc_wait_ld();
+      for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + 32 * c, sr[c]);
+      ptx::tc_wait_ld_regs(sr[0]);
+      ptx::reg_fence32(sr[1]);
+      ptx::reg_fence32(sr[2]);
+      ptx::reg_fence32(sr[3]);
+
+      // Row maximum of x = S * g_K(chunk) * scale * log2(e) (masked keys -inf).
+      float mx;
+      if (uni) {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float s0 = __uint_as_float(r[2 * i]), s1 = __uint_as_float(r[2 * i + 1]);
-            if (i & 1) mb = ptx::fmax3(mb, s0, s1); else ma = ptx::fmax3(ma, s0, s1);
-            pk[16 * c + i] = ptx::f32x2_to_f16x2(ptx::ex2(fmaf(s0, ck, mneg)), ptx::ex2(fmaf(s1, ck, mneg)));
-            if (i & 1) lb = ptx::add_f16x2_f32(lb, pk[16 * c + i]);
-            else la = ptx::add_f16x2_f32(la, pk[16 * c + i]);
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            m4[c] = ptx::fmax3(m4[c], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
+        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * ck;
+      } else {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int jj = 32 * c + i;
+            m4[c] = fmaxf(m4[c], jj < info.x ? __uint_as_float(sr[c][i]) * colK[jj] * q_unscale : -INFINITY);
           }
-        }
-        redo = __any_sync(0xFFFFFFFFu, fmaxf(ma, mb) * ck > m_run + 8.0f);
-        if (!redo) l_run += (la + lb) / cv;
+        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
-      if (redo) {
-        // General case (first tile, a tile across chunk boundaries or with masked keys, an
-        // all-zero V chunk, or a jump of the maximum): exact row maximum first.
-        float mx;
-        {
-          float ma = -INFINITY, mb = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tS + 32 * c, r);
-            ptx::tc_wait_ld();
-            if (info.y) {
-#pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                ma = ptx::fmax3(ma, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-                mb = ptx::fmax3(mb, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int jj = 32 * c + i;
-                ma = fmaxf(ma, jj < info.x ? __uint_as_float(r[i]) * colK[jj] * q_unscale : -INFINITY);
-              }
-            }
-          }
-          mx = info.y ? fmaxf(ma, mb) * ck : fmaxf(ma, mb);
-        }
-        // Lazy rescale: a row moves its running max only when it grew by more than 2^8.  The O
-        // rescale uses warp-collective TMEM accesses, so it runs for the whole warp when any
-        // row of the warp moved (alpha = 1 for the rows that did not).
-        const bool moved = mx > m_run + 8.0f;
-        float alpha = 1.0f;
-        if (moved) {
-          alpha = ptx::ex2(m_run - mx);
-          l_run *= alpha;
-          m_run = mx;
-        }
-        if (j > 0 && __any_sync(0xFFFFFFFFu, moved)) {
+      // Lazy rescale: the reference m only moves (to a whole number, so the rescale is an exact
+      // power of two) when the row maximum exceeds it by more than 2^8.  The O rescale uses
+      // warp-collective TMEM accesses, so it runs for the whole warp when any row moved
+      // (alpha = 1 for the rows that did not).
+      const bool grow = mx > m_run + 8.0f;
+      if (__any_sync(0xFFFFFFFFu, grow)) {
+        const float m_new = grow ? ceilf(mx) : m_run;
+        const float alpha = grow ? ptx::ex2(m_run - m_new) : 1.0f;  // 0 while m is -inf
+        l_run *= alpha;
+        m_run = m_new;
+        if (j > 0) {  // O holds tiles < j; PV(j - 1) is complete (it precedes QK(j))
           ok = waitw(bar(C::bODone + qt), (j - 1) & 1, abort_flag, p.status);
           if (!ok) break;
           ptx::tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tO + 32 * c, r);
-            ptx::tc_wait_ld();
+          for (int oc = 0; oc < 8; ++oc) {  // 16 columns at a time: the S row stays in registers
+            uint32_t o[16];
+            ptx::tmem_ld16_wait(tO + 16 * oc, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            ptx::tmem_st32(tO + 32 * c, r);
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            ptx::tmem_st16p(tO + 16 * oc, o);
           }
-        }
-        float la = 0.0f, lb = 0.0f;
-        if (info.y) {
-          // a key of an all-zero V chunk (cv = 0) adds 0 to O and its p to l
-          const float cv = colV[0];
-          const float mneg = (cv > 0.0f ? log2f(cv) : 0.0f) - m_run;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tS + 32 * c, r);
-            ptx::tc_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float p0 = ptx::ex2(fmaf(__uint_as_float(r[2 * i]), ck, mneg));
-              const float p1 = ptx::ex2(fmaf(__uint_as_float(r[2 * i + 1]), ck, mneg));
-              if (cv > 0.0f) {
-                pk[16 * c + i] = ptx::f32x2_to_f16x2(p0, p1);
-                if (i & 1) lb = ptx::add_f16x2_f32(lb, pk[16 * c + i]);
-                else la = ptx::add_f16x2_f32(la, pk[16 * c + i]);
-              } else {
-                pk[16 * c + i] = 0u;
-                la += p0;
-                lb += p1;
-              }
-            }
-          }
-          l_run += cv > 0.0f ? (la + lb) / cv : la + lb;
-        } else {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tS + 32 * c, r);
-            ptx::tc_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int j0 = 32 * c + 2 * i;
-              const float x0 = j0 < info.x ? __uint_as_float(r[2 * i]) * colK[j0] * q_unscale : -INFINITY;
-              const float x1 =
-                  j0 + 1 < info.x ? __uint_as_float(r[2 * i + 1]) * colK[j0 + 1] * q_unscale : -INFINITY;
-              const float p0 = ptx::ex2(x0 - m_run), p1 = ptx::ex2(x1 - m_run);
-              const float cv0 = colV[j0], cv1 = colV[j0 + 1];
-              const uint32_t w = ptx::f32x2_to_f16x2(p0 * cv0, p1 * cv1);
-              pk[16 * c + i] = w;
-              const float t0 = __half2float(__ushort_as_half(static_cast<uint16_t>(w & 0xFFFFu)));
-              const float t1 = __half2float(__ushort_as_half(static_cast<uint16_t>(w >> 16)));
-              la += cv0 > 0.0f ? t0 / cv0 : p0;
-              lb += cv1 > 0.0f ? t1 / cv1 : p1;
-            }
-          }
-          l_run += la + lb;
         }
       }
+
+      // P~ = 2^(x - m) * cv (cv = g_V(chunk) / max g_V), rounded to fp16 pairs and stored over
+      // S's first 64 columns (chunk c -> P columns [16c, 16c + 16)).  The row sum adds the same
+      // rounded values divided by cv, so the rounding largely cancels in O / l; a key of an
+      // all-zero V chunk (cv = 0) adds 0 to O and its p to l.
+      float la = 0.0f, lb = 0.0f;
+      if (uni) {
+        const float mneg = log2f(colV[0]) - m_run;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) ptx::tmem_st16p(tS + 16 * c, &pk[16 * c]);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            pk[i] = ptx::f32x2_to_f16x2(ptx::ex2(fmaf(__uint_as_float(sr[c][2 * i]), ck, mneg)),
+                                        ptx::ex2(fmaf(__uint_as_float(sr[c][2 * i + 1]), ck, mneg)));
+            if (i & 1) lb = ptx::add_f16x2_f32(lb, pk[i]);
+            else la = ptx::add_f16x2_f32(la, pk[i]);
+          }
+          ptx::tmem_st16p(tS + 16 * c, pk);
+        }
+        l_run += (la + lb) / colV[0];
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int j0 = 32 * c + 2 * i;
+            const float x0 = j0 < info.x ? __uint_as_float(sr[c][2 * i]) * colK[j0] * q_unscale : -INFINITY;
+            const float x1 =
+                j0 + 1 < info.x ? __uint_as_float(sr[c][2 * i + 1]) * colK[j0 + 1] * q_unscale : -INFINITY;
+            const float p0 = x0 == -INFINITY ? 0.0f : ptx::ex2(x0 - m_run);
+            const float p1 = x1 == -INFINITY ? 0.0f : ptx::ex2(x1 - m_run);
+            const float cv0 = colV[j0], cv1 = colV[j0 + 1];
+            pk[i] = ptx::f32x2_to_f16x2(p0 * cv0, p1 * cv1);
+            const float t0 = __half2float(__ushort_as_half(static_cast<uint16_t>(pk[i] & 0xFFFFu)));
+            const float t1 = __half2float(__ushort_as_half(static_cast<uint16_t>(pk[i] >> 16)));
+            la += cv0 > 0.0f ? t0 / cv0 : p0;
+            lb += cv1 > 0.0f ? t1 / cv1 : p1;
+          }
+          ptx::tmem_st16p(tS + 16 * c, pk);
+        }
+        l_run += la + lb;
+      }
       ptx::tc_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
@@ -518,7 +499,9 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
         }
       }
     }
-  } else if (warp == C::kProducerWarp) {
+  } else {
+  if constexpr (QT == 2) ptx::setmaxnreg_dec<80>();
+  if (warp == C::kProducerWarp) {
     // ============================================================ TMA producer
     if (lane == 0) {
       ptx::prefetch_tmap(&tmap_q);
@@ -559,64 +542,69 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
     __syncwarp();
   } else if (warp == C::kMmaWarp) {
     // ============================================================ MMA issuer
-    if (lane == 0) {
-      // kind::f16 instruction descriptors: fp16 x fp16 -> fp32; M = 128; N = 128.
-      constexpr uint32_t kIdescQK = (1u << 4) |  // A = Q and B = K^ both K-major
-                                    (static_cast<uint32_t>(BN >> 3) << 17) |
-                                    (static_cast<uint32_t>(BM >> 4) << 24);
-      constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) |  // B = V^ MN-major
-                                    (static_cast<uint32_t>(D >> 3) << 17) |
-                                    (static_cast<uint32_t>(BM >> 4) << 24);
-      auto issue_qk = [&](int q, int st) {
-        const uint32_t sQ = sbase + C::oQ + q * TILE16;
-        const uint32_t sK = sbase + C::oK + st * TILE16;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * HALF16 + (kk & 3) * 32;
-          ptx::mma_ss(tmem + q * BN, ptx::smem_desc_sw128(sQ + koff, 16, 1024),
-                      ptx::smem_desc_sw128(sK + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
-        }
-        ptx::mma_commit(bar(C::bSFull + q));
-      };
-      bool ok = wait1(bar(C::bQReady), 0, abort_flag, p.status) && p.n_tiles > 0 &&
-                wait1(bar(C::bKFull + 0), 0, abort_flag, p.status);
-      if (ok) {
-        ptx::tc_fence_after();
-        for (int q = 0; q < QT; ++q) issue_qk(q, 0);
+    // The whole warp runs this loop with warp-uniform values; one elected lane issues each
+    // tcgen05 instruction.
+    // kind::f16 instruction descriptors: fp16 x fp16 -> fp32; M = 128; N = 128.
+    constexpr uint32_t kIdescQK = (1u << 4) |  // A = Q and B = K^ both K-major
+                                  (static_cast<uint32_t>(BN >> 3) << 17) |
+                                  (static_cast<uint32_t>(BM >> 4) << 24);
+    constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) |  // B = V^ MN-major
+                                  (static_cast<uint32_t>(D >> 3) << 17) |
+                                  (static_cast<uint32_t>(BM >> 4) << 24);
+    // Shared-memory descriptors are built once; a K step only advances the 14-bit start address
+    // field (address >> 4), so each MMA costs one add per operand.
+    const uint64_t dQ0 = ptx::smem_desc_sw128(sbase + C::oQ, 16, 1024);
+    const uint64_t dK0 = ptx::smem_desc_sw128(sbase + C::oK, 16, 1024);
+    const uint64_t dV0 = ptx::smem_desc_sw128(sbase + C::oV, HALF16, 1024);
+    auto issue_qk = [&](int q, int st) {
+      const uint64_t dQ = dQ0 + static_cast<uint64_t>((q * TILE16) >> 4);
+      const uint64_t dK = dK0 + static_cast<uint64_t>((st * TILE16) >> 4);
+      const uint32_t tS = tmem + q * BN;
+#pragma unroll 1  // kept rolled: the MMA warp runs on an 80-register budget
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * HALF16 + (kk & 3) * 32) >> 4);
+        ptx::mma_ss_w(tS, dQ + koff, dK + koff, kIdescQK, kk > 0 ? 1u : 0u);
       }
-      // Per KV tile j: PV(q, j) as soon as softmax q has written P(q, j), then QK(q, j + 1) into
-      // the same S columns; the two query tiles alternate so the tensor core always has the
-      // other tile's work while one softmax runs.
-      for (int j = 0; j < p.n_tiles && ok; ++j) {
-        const int st = j % NST;
-        const uint32_t sV = sbase + C::oV + st * TILE16;
-        for (int q = 0; q < QT && ok; ++q) {
-          ok = wait1(bar(C::bPFull + q), j & 1, abort_flag, p.status);
-          if (ok && q == 0) ok = wait1(bar(C::bVFull + st), (j / NST) & 1, abort_flag, p.status);
-          if (!ok) break;
-          ptx::tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            ptx::mma_ts(tmem + QT * BN + q * D, tmem + q * BN + kk * 8,
-                        ptx::smem_desc_sw128(sV + kk * 2048, HALF16, 1024), kIdescPV,
-                        (j > 0 || kk > 0) ? 1u : 0u);
-          ptx::mma_commit(bar(C::bODone + q));
-          if (q == QT - 1) ptx::mma_commit(bar(C::bKvEmpty + st));
-          if (j + 1 < p.n_tiles) {
-            const int st1 = (j + 1) % NST;
-            if (q == 0) {
-              ok = wait1(bar(C::bKFull + st1), ((j + 1) / NST) & 1, abort_flag, p.status);
-              if (!ok) break;
-              ptx::tc_fence_after();
-            }
-            issue_qk(q, st1);
-          }
-        }
-      }
-      // every MMA issued so far completes before the drain barrier's phase 0
-      ptx::mma_commit(bar(C::bDrain));
-      wait_drain(bar(C::bDrain), 0, p.status);
+      ptx::mma_commit_w(bar(C::bSFull + q));
+    };
+    bool ok = waitw(bar(C::bQReady), 0, abort_flag, p.status) && p.n_tiles > 0 &&
+              waitw(bar(C::bKFull + 0), 0, abort_flag, p.status);
+    if (ok) {
+      ptx::tc_fence_after();
+      for (int q = 0; q < QT; ++q) issue_qk(q, 0);
     }
+    // Per KV tile j: PV(q, j) as soon as softmax q has written P(q, j), then QK(q, j + 1) into the
+    // same S columns; the two query tiles alternate so the tensor core always has the other
+    // tile's work while one softmax runs.
+    for (int j = 0; j < p.n_tiles && ok; ++j) {
+      const int st = j % NST;
+      for (int q = 0; q < QT && ok; ++q) {
+        ok = waitw(bar(C::bPFull + q), j & 1, abort_flag, p.status);
+        if (ok && q == 0) ok = waitw(bar(C::bVFull + st), (j / NST) & 1, abort_flag, p.status);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const uint64_t dV = dV0 + static_cast<uint64_t>((st * TILE16) >> 4);
+        const uint32_t tO = tmem + QT * BN + q * D, tP = tmem + q * BN;
+#pragma unroll 1
+        for (int kk = 0; kk < BN / 16; ++kk)
+          ptx::mma_ts_w(tO, tP + kk * 8, dV + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescPV,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+        ptx::mma_commit_w(bar(C::bODone + q));
+        if (q == QT - 1) ptx::mma_commit_w(bar(C::bKvEmpty + st));
+        if (j + 1 < p.n_tiles) {
+          const int st1 = (j + 1) % NST;
+          if (q == 0) {
+            ok = waitw(bar(C::bKFull + st1), ((j + 1) / NST) & 1, abort_flag, p.status);
+            if (!ok) break;
+            ptx::tc_fence_after();
+          }
+          issue_qk(q, st1);
+        }
+      }
+    }
+    // every MMA issued so far completes before the drain barrier's phase 0
+    ptx::mma_commit_w(bar(C::bDrain));
+    if (lane == 0) wait_drain(bar(C::bDrain), 0, p.status);
     __syncwarp();
   } else {
     // ============================================================ dequant warps
@@ -635,8 +623,8 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
         ok = waitw(bar(C::bPkFull + slot), (pk / NPK) & 1, abort_flag, p.status);
         if (!ok) break;
         const uint8_t* src = smem + C::oPK + slot * PK_BYTES;
-        dequant_tile(src, smem + (t == 0 ? C::oK : C::oV) + st * TILE16, n, dt);
-        if (t == 0) {
+        dequant_tile<C::kDequantThreads>(src, smem + (t == 0 ? C::oK : C::oV) + st * TILE16, n, dt);
+        if (t == 0 && dt < BN) {  // per-column tables: one thread per key of the tile
           float* colK = reinterpret_cast<float*>(smem + C::oCol + st * 2 * BN * 4);
           const bool valid = dt < n;
           const int c = valid ? (key0 + dt) / p.Lc : 0;
@@ -655,6 +643,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
         }
       }
     }
+  }
   }
 
   ptx::tc_fence_before();
