@@ -46,11 +46,21 @@ constexpr int BN = 128;  // keys per KV tile
 constexpr int D = kHeadDim;
 constexpr int NST = 2;   // stages of dequantised K / V tiles
 constexpr int NPK = 3;   // slots of packed data (K and V tiles alternate)
+constexpr int NCT = 4;   // slots of per-tile column tables
+constexpr int kMaxTabChunks = 256;  // chunk scales staged in shared memory up to this many slots
 constexpr int PK_CODES = BN * kCodeBytes;               // 8192
 constexpr int PK_BYTES = PK_CODES + BN * kScaleBytes;   // 9216
 constexpr int TILE16 = BN * D * 2;                      // one 128 x 128 16-bit operand tile
 constexpr int HALF16 = TILE16 / 2;                      // 128 rows x 64 elements (128 B rows)
 constexpr int MAX_RUNS = 4;
+#ifndef NVFP4KV_EXP2_EMUL
+#define NVFP4KV_EXP2_EMUL 0
+#endif
+constexpr int kExp2Emul = NVFP4KV_EXP2_EMUL;  // 0: every exponent on the MUFU
+#ifndef NVFP4KV_TURNS
+#define NVFP4KV_TURNS 0
+#endif
+constexpr bool kTurns = NVFP4KV_TURNS != 0;  // the two softmax warpgroups take turns
 
 template <int QT>
 struct Cfg {
@@ -60,6 +70,7 @@ struct Cfg {
   static constexpr int kDequantWarp0 = kSoftmaxWarps + 2;
   static constexpr int kDequantWarps = 6;  // 2 in the producer/MMA warpgroup + one full warpgroup
   static constexpr int kDequantThreads = 32 * kDequantWarps;
+  static_assert(kDequantThreads == 192, "dequant_tile deals blocks to 192 threads");
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 2 + kDequantWarps);  // whole warpgroups
   static constexpr uint32_t kTmemCols = QT == 1 ? 256 : 512;
   // shared memory map (bytes from a 1024-aligned base)
@@ -67,10 +78,14 @@ struct Cfg {
   static constexpr int oK = oQ + QT * TILE16;
   static constexpr int oV = oK + NST * TILE16;
   static constexpr int oPK = oV + NST * TILE16;
-  static constexpr int oCol = oPK + NPK * PK_BYTES;      // per stage: colK[BN], colV[BN] (fp32)
-  static constexpr int oInfo = oCol + NST * 2 * BN * 4;  // per stage: int4 {n_valid, uniform}
-  static constexpr int oRed = oInfo + NST * 16;          // per Q tile: 4 warp maxima
-  static constexpr int oBar = oRed + QT * 16;
+  // Per-tile column tables colK[BN], colV[BN] (fp32) and int4 {n_valid, uniform}, in NCT slots:
+  // the K stage of tile j is refilled once the QKs of tile j - NST are done, while the softmax
+  // warps may still read the tables of tiles j - NST and j - NST + 1.
+  static constexpr int oCol = oPK + NPK * PK_BYTES;
+  static constexpr int oInfo = oCol + NCT * 2 * BN * 4;
+  static constexpr int oRed = oInfo + NCT * 16;          // per Q tile: 4 warp maxima
+  static constexpr int oTab = oRed + QT * 16;            // per chunk slot: {g_K * scale, g_V / max g_V}
+  static constexpr int oBar = oTab + kMaxTabChunks * 8;
   // barrier indices
   static constexpr int bQFull = 0;
   static constexpr int bQReady = 1;
@@ -78,12 +93,14 @@ struct Cfg {
   static constexpr int bPkEmpty = bPkFull + NPK;
   static constexpr int bKFull = bPkEmpty + NPK;
   static constexpr int bVFull = bKFull + NST;
-  static constexpr int bKvEmpty = bVFull + NST;
-  static constexpr int bSFull = bKvEmpty + NST;
+  static constexpr int bKEmpty = bVFull + NST;  // K stage read by every QK of its tile
+  static constexpr int bVEmpty = bKEmpty + NST;  // V stage read by every PV of its tile
+  static constexpr int bSFull = bVEmpty + NST;
   static constexpr int bPFull = bSFull + QT;
   static constexpr int bODone = bPFull + QT;
   static constexpr int bDrain = bODone + QT;
-  static constexpr int kNumBars = bDrain + 1;
+  static constexpr int bTok = bDrain + 1;  // softmax turn: [0] tile 0 -> tile 1, [1] tile 1 -> tile 0
+  static constexpr int kNumBars = bTok + 2;
   static constexpr int oMisc = oBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag
   static constexpr int kSmemBytes = oMisc + 16 + 1024;  // + slack for 1024-B alignment
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -188,50 +205,52 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
 
 // Dequantise one packed tile (codes + E4M3 scales of BN keys) into a 128B-swizzled [key][d]
 // operand tile of fp16 values, code * scale (exact: <= 6 significant bits, 2^-10 .. 2688).
-// The 1024 16-element blocks of a tile are dealt round-robin to NT threads, three at a time
-// with all their shared-memory loads issued first (one scale conversion per block).
-template <int NT>
+// Thread dt of NT = 192 owns the 16-element block blk = dt % 8 of keys dt / 8 + 24 * it: 192 is a
+// multiple of 8 (the block, the swizzle phase key % 8 and the store order are fixed per thread)
+// and of 24 rows of the operand tile (every address is a per-thread base plus a constant).  All
+// shared-memory loads are issued first.  A 16-byte warp store is served in phases of 8 lanes (one
+// key, all eight blocks): lanes of the second 64-element half store their odd chunk first, so the
+// 8 lanes of a phase hit 8 distinct banks.  Keys >= n (past the run's end) are written as zeros.
+template <bool kFull>
 __device__ __forceinline__ void dequant_tile(const uint8_t* pk, uint8_t* dst, int n, int dt) {
-  constexpr int kPer = (1024 + NT - 1) / NT;  // blocks per thread, rounded up
-#pragma unroll 1
-  for (int base = 0; base < kPer; base += 3) {
-    uint2 w[3];
-    uint32_t sb[3];
+  constexpr int NT = 192, KS = NT / 8;  // 24 keys per pass
+  constexpr int kIt = (BN + KS - 1) / KS;  // 6 passes; the last one only for dt < 64
+  const int blk = dt & 7, kq = dt >> 3;
+  const bool swap = blk >= 4;
+  const int c0 = (blk & 3) * 2;
+  const uint8_t* csrc = pk + kq * kCodeBytes + blk * 8;
+  const uint8_t* ssrc = pk + PK_CODES + kq * kScaleBytes + blk;
+  uint8_t* const row = dst + (blk >> 2) * HALF16 + kq * 128;
+  uint8_t* const dA = row + (((c0 + (swap ? 1 : 0)) ^ (kq & 7)) << 4);  // first store
+  uint8_t* const dB = row + (((c0 + (swap ? 0 : 1)) ^ (kq & 7)) << 4);
+  const bool tail = kq + KS * (kIt - 1) < BN;  // this thread has a sixth key
+  uint2 w[kIt];
+  uint32_t sb[kIt];
 #pragma unroll
-    for (int u = 0; u < 3; ++u) {
-      const int job = (base + u) * NT + dt;
-      if (base + u < kPer && job < 1024) {
-        const int key = job >> 3, blk = job & 7;
-        w[u] = *reinterpret_cast<const uint2*>(pk + key * kCodeBytes + blk * 8);
-        sb[u] = pk[PK_CODES + key * kScaleBytes + blk];
-      }
+  for (int it = 0; it < kIt; ++it) {
+    if (it < kIt - 1 || tail) {
+      w[it] = *reinterpret_cast<const uint2*>(csrc + it * KS * kCodeBytes);
+      sb[it] = ssrc[it * KS * kScaleBytes];
     }
+  }
 #pragma unroll
-    for (int u = 0; u < 3; ++u) {
-      const int job = (base + u) * NT + dt;
-      if (base + u >= kPer || job >= 1024) continue;
-      const int key = job >> 3, blk = job & 7;
-      const uint32_t s2 = ptx::e4m3_to_f16x2_bcast(sb[u]);
-      uint32_t h[4], g[4];
-      ptx::e2m1x8_to_f16x8(w[u].x, h);
-      ptx::e2m1x8_to_f16x8(w[u].y, g);
-      uint4 o0 = make_uint4(ptx::hmul2_u32(h[0], s2), ptx::hmul2_u32(h[1], s2), ptx::hmul2_u32(h[2], s2),
-                            ptx::hmul2_u32(h[3], s2));
-      uint4 o1 = make_uint4(ptx::hmul2_u32(g[0], s2), ptx::hmul2_u32(g[1], s2), ptx::hmul2_u32(g[2], s2),
-                            ptx::hmul2_u32(g[3], s2));
-      if (key >= n) {  // past the run's last key: zero rows (P is 0 there, 0 * 0 stays 0)
-        o0 = make_uint4(0, 0, 0, 0);
-        o1 = o0;
-      }
-      // 16-byte chunks c0, c0 + 1 of the 128-byte row (64 elements per half).  A 16-byte warp
-      // store is served in phases of 8 lanes (one key, both halves of the row); lanes of the
-      // second half store their odd chunk first, so the 8 lanes of a phase hit 8 distinct banks.
-      const int c0 = (blk * 2) & 7;
-      const bool swap = blk >= 4;
-      uint8_t* row = dst + (blk >> 2) * HALF16 + key * 128;
-      *reinterpret_cast<uint4*>(row + (((c0 + (swap ? 1 : 0)) ^ (key & 7)) << 4)) = swap ? o1 : o0;
-      *reinterpret_cast<uint4*>(row + (((c0 + (swap ? 0 : 1)) ^ (key & 7)) << 4)) = swap ? o0 : o1;
+  for (int it = 0; it < kIt; ++it) {
+    if (it == kIt - 1 && !tail) break;
+    const uint32_t s2 = ptx::e4m3_to_f16x2_bcast(sb[it]);
+    const uint32_t first = swap ? w[it].y : w[it].x, second = swap ? w[it].x : w[it].y;
+    uint32_t h[4], g[4];
+    ptx::e2m1x8_to_f16x8(first, h);
+    ptx::e2m1x8_to_f16x8(second, g);
+    uint4 oA = make_uint4(ptx::hmul2_u32(h[0], s2), ptx::hmul2_u32(h[1], s2), ptx::hmul2_u32(h[2], s2),
+                          ptx::hmul2_u32(h[3], s2));
+    uint4 oB = make_uint4(ptx::hmul2_u32(g[0], s2), ptx::hmul2_u32(g[1], s2), ptx::hmul2_u32(g[2], s2),
+                          ptx::hmul2_u32(g[3], s2));
+    if (!kFull && kq + KS * it >= n) {
+      oA = make_uint4(0, 0, 0, 0);
+      oB = oA;
     }
+    *reinterpret_cast<uint4*>(dA + it * KS * 128) = oA;
+    *reinterpret_cast<uint4*>(dB + it * KS * 128) = oB;
   }
 }
 
@@ -263,7 +282,8 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
     for (int i = 0; i < NST; ++i) {
       ptx::mbar_init(bar(C::bKFull + i), C::kDequantWarps);
       ptx::mbar_init(bar(C::bVFull + i), C::kDequantWarps);
-      ptx::mbar_init(bar(C::bKvEmpty + i), 1);
+      ptx::mbar_init(bar(C::bKEmpty + i), 1);
+      ptx::mbar_init(bar(C::bVEmpty + i), 1);
     }
     for (int q = 0; q < QT; ++q) {
       ptx::mbar_init(bar(C::bSFull + q), 1);
@@ -271,6 +291,8 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       ptx::mbar_init(bar(C::bODone + q), 1);
     }
     ptx::mbar_init(bar(C::bDrain), 1);
+    ptx::mbar_init(bar(C::bTok + 0), 4);
+    ptx::mbar_init(bar(C::bTok + 1), 4);
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::fence_proxy_async_smem();
@@ -348,10 +370,18 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       const int st = j % NST;
       ok = waitw(bar(C::bSFull + qt), j & 1, abort_flag, p.status) &&
            waitw(bar(C::bKFull + st), (j / NST) & 1, abort_flag, p.status);
+      // With two query tiles the two softmax warpgroups take turns (tile 0 of KV tile j, tile 1 of
+      // j, tile 0 of j + 1, ...): each runs with the SM's exponent and conversion units to itself
+      // while the tensor core works on the other tile's products.
+      if (QT == 2 && kTurns && ok) {
+        if (qt == 1) ok = waitw(bar(C::bTok + 0), j & 1, abort_flag, p.status);
+        else if (j > 0) ok = waitw(bar(C::bTok + 1), (j - 1) & 1, abort_flag, p.status);
+      }
       if (!ok) break;
       ptx::tc_fence_after();
-      const int4 info = *reinterpret_cast<const int4*>(smem + C::oInfo + 16 * st);
-      const float* colK = reinterpret_cast<const float*>(smem + C::oCol + st * 2 * BN * 4);
+      const int ct = j % NCT;
+      const int4 info = *reinterpret_cast<const int4*>(smem + C::oInfo + 16 * ct);
+      const float* colK = reinterpret_cast<const float*>(smem + C::oCol + ct * 2 * BN * 4);
       const float* colV = colK + BN;
       const float ck = colK[0] * q_unscale;
       // A tile inside one chunk with every key valid and a nonzero V scale takes the uniform path
@@ -370,13 +400,19 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       // Row maximum of x = S * g_K(chunk) * scale * log2(e) (masked keys -inf).
       float mx;
       if (uni) {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float m8[8];  // eight independent max chains
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; i += 2)
-            m4[c] = ptx::fmax3(m4[c], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
-        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * ck;
+          for (int i = 0; i < 32; i += 4) {
+            m8[2 * c] = ptx::fmax3(m8[2 * c], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
+            m8[2 * c + 1] =
+                ptx::fmax3(m8[2 * c + 1], __uint_as_float(sr[c][i + 2]), __uint_as_float(sr[c][i + 3]));
+          }
+        mx = fmaxf(ptx::fmax3(m8[0], m8[1], m8[2]), ptx::fmax3(m8[3], m8[4], ptx::fmax3(m8[5], m8[6], m8[7]))) *
+             ck;
       } else {
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -419,19 +455,27 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       // all-zero V chunk (cv = 0) adds 0 to O and its p to l.
       float la = 0.0f, lb = 0.0f;
       if (uni) {
+        // x = S * ck + log2(cv) - m in packed pairs; one exponent in 2 * kExp2Emul is taken on the
+        // FMA pipe (ex2_poly3) to relieve the MUFU; eight independent row-sum chains.
         const float mneg = log2f(colV[0]) - m_run;
+        float l8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) l8[k] = 0.0f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            pk[i] = ptx::f32x2_to_f16x2(ptx::ex2(fmaf(__uint_as_float(sr[c][2 * i]), ck, mneg)),
-                                        ptx::ex2(fmaf(__uint_as_float(sr[c][2 * i + 1]), ck, mneg)));
-            if (i & 1) lb = ptx::add_f16x2_f32(lb, pk[i]);
-            else la = ptx::add_f16x2_f32(la, pk[i]);
+            float x0, x1;
+            ptx::ffma2(x0, x1, __uint_as_float(sr[c][2 * i]), __uint_as_float(sr[c][2 * i + 1]), ck, mneg);
+            const bool emul = kExp2Emul > 0 && (i % (kExp2Emul > 0 ? kExp2Emul : 1)) == kExp2Emul - 1;
+            pk[i] = ptx::f32x2_to_f16x2(emul ? ptx::ex2_poly3(x0) : ptx::ex2(x0), ptx::ex2(x1));
+            l8[i & 7] = ptx::add_f16x2_f32(l8[i & 7], pk[i]);
           }
           ptx::tmem_st16p(tS + 16 * c, pk);
         }
+        la = (l8[0] + l8[1]) + (l8[2] + l8[3]);
+        lb = (l8[4] + l8[5]) + (l8[6] + l8[7]);
         l_run += (la + lb) / colV[0];
       } else {
 #pragma unroll
@@ -455,6 +499,10 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
           ptx::tmem_st16p(tS + 16 * c, pk);
         }
         l_run += la + lb;
+      }
+      if (QT == 2 && kTurns) {
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(C::bTok + qt));
       }
       ptx::tc_wait_st();
       ptx::tc_fence_before();
@@ -552,7 +600,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
                                   (static_cast<uint32_t>(D >> 3) << 17) |
                                   (static_cast<uint32_t>(BM >> 4) << 24);
     // Shared-memory descriptors are built once; a K step only advances the 14-bit start address
-    // field (address >> 4), so each MMA costs one add per operand.
+    // field (address >> 4).
     const uint64_t dQ0 = ptx::smem_desc_sw128(sbase + C::oQ, 16, 1024);
     const uint64_t dK0 = ptx::smem_desc_sw128(sbase + C::oK, 16, 1024);
     const uint64_t dV0 = ptx::smem_desc_sw128(sbase + C::oV, HALF16, 1024);
@@ -560,11 +608,8 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       const uint64_t dQ = dQ0 + static_cast<uint64_t>((q * TILE16) >> 4);
       const uint64_t dK = dK0 + static_cast<uint64_t>((st * TILE16) >> 4);
       const uint32_t tS = tmem + q * BN;
-#pragma unroll 1  // kept rolled: the MMA warp runs on an 80-register budget
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * HALF16 + (kk & 3) * 32) >> 4);
-        ptx::mma_ss_w(tS, dQ + koff, dK + koff, kIdescQK, kk > 0 ? 1u : 0u);
-      }
+      // one asm block of eight MMAs: a rolled loop issued an MMA only every ~80 cycles
+      ptx::mma_qk8_w(tS, dQ, dK, kIdescQK, 0u);
       ptx::mma_commit_w(bar(C::bSFull + q));
     };
     bool ok = waitw(bar(C::bQReady), 0, abort_flag, p.status) && p.n_tiles > 0 &&
@@ -572,6 +617,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
     if (ok) {
       ptx::tc_fence_after();
       for (int q = 0; q < QT; ++q) issue_qk(q, 0);
+      ptx::mma_commit_w(bar(C::bKEmpty + 0));
     }
     // Per KV tile j: PV(q, j) as soon as softmax q has written P(q, j), then QK(q, j + 1) into the
     // same S columns; the two query tiles alternate so the tensor core always has the other
@@ -585,12 +631,9 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
         ptx::tc_fence_after();
         const uint64_t dV = dV0 + static_cast<uint64_t>((st * TILE16) >> 4);
         const uint32_t tO = tmem + QT * BN + q * D, tP = tmem + q * BN;
-#pragma unroll 1
-        for (int kk = 0; kk < BN / 16; ++kk)
-          ptx::mma_ts_w(tO, tP + kk * 8, dV + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescPV,
-                        (j > 0 || kk > 0) ? 1u : 0u);
+        ptx::mma_pv8_w(tO, tP, dV, kIdescPV, j > 0 ? 1u : 0u);
         ptx::mma_commit_w(bar(C::bODone + q));
-        if (q == QT - 1) ptx::mma_commit_w(bar(C::bKvEmpty + st));
+        if (q == QT - 1) ptx::mma_commit_w(bar(C::bVEmpty + st));
         if (j + 1 < p.n_tiles) {
           const int st1 = (j + 1) % NST;
           if (q == 0) {
@@ -599,6 +642,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
             ptx::tc_fence_after();
           }
           issue_qk(q, st1);
+          if (q == QT - 1) ptx::mma_commit_w(bar(C::bKEmpty + st1));
         }
       }
     }
@@ -610,29 +654,44 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
     // ============================================================ dequant warps
     const int dt = threadIdx.x - C::kDequantWarp0 * 32;
     const float inv_gv = 1.0f / max_visible_gv(p, bh);
+    // The per-chunk FP32 scales of this (b, h), staged once, so the per-tile column tables are
+    // built from shared memory.
+    const float2* gtab = reinterpret_cast<const float2*>(smem + C::oTab);
+    const bool use_tab = p.C <= kMaxTabChunks;
+    if (use_tab)
+      for (int c = dt; c < p.C; c += C::kDequantThreads)
+        reinterpret_cast<float2*>(smem + C::oTab)[c] =
+            make_float2(p.k_g[bh * p.C + c] * p.scale_log2, p.v_g[bh * p.C + c] * inv_gv);
+    ptx::named_bar(3, C::kDequantThreads);
     bool ok = true;
     for (int j = 0; j < p.n_tiles && ok; ++j) {
       const int st = j % NST;
-      if (j >= NST) ok = waitw(bar(C::bKvEmpty + st), ((j / NST) - 1) & 1, abort_flag, p.status);
-      if (!ok) break;
       int key0, n;
       tile_keys(p, j, key0, n);
       for (int t = 0; t < 2 && ok; ++t) {
+        // the stage's previous tile (j - NST) is done with it: K after its QKs, V after its PVs
+        if (j >= NST) ok = waitw(bar((t == 0 ? C::bKEmpty : C::bVEmpty) + st), ((j / NST) - 1) & 1, abort_flag, p.status);
+        if (!ok) break;
         const int pk = 2 * j + t;
         const int slot = pk % NPK;
         ok = waitw(bar(C::bPkFull + slot), (pk / NPK) & 1, abort_flag, p.status);
         if (!ok) break;
         const uint8_t* src = smem + C::oPK + slot * PK_BYTES;
-        dequant_tile<C::kDequantThreads>(src, smem + (t == 0 ? C::oK : C::oV) + st * TILE16, n, dt);
+        uint8_t* dst = smem + (t == 0 ? C::oK : C::oV) + st * TILE16;
+        if (n == BN) dequant_tile<true>(src, dst, n, dt);
+        else dequant_tile<false>(src, dst, n, dt);
         if (t == 0 && dt < BN) {  // per-column tables: one thread per key of the tile
-          float* colK = reinterpret_cast<float*>(smem + C::oCol + st * 2 * BN * 4);
+          float* colK = reinterpret_cast<float*>(smem + C::oCol + (j % NCT) * 2 * BN * 4);
           const bool valid = dt < n;
           const int c = valid ? (key0 + dt) / p.Lc : 0;
-          colK[dt] = valid ? p.k_g[bh * p.C + c] * p.scale_log2 : 0.0f;
-          colK[BN + dt] = valid ? p.v_g[bh * p.C + c] * inv_gv : 0.0f;
+          const float2 g = !valid ? make_float2(0.0f, 0.0f)
+                           : use_tab ? gtab[c]
+                                     : make_float2(p.k_g[bh * p.C + c] * p.scale_log2, p.v_g[bh * p.C + c] * inv_gv);
+          colK[dt] = g.x;
+          colK[BN + dt] = g.y;
           if (dt == 0) {
             const int uniform = (n == BN) && (key0 / p.Lc == (key0 + BN - 1) / p.Lc);
-            *reinterpret_cast<int4*>(smem + C::oInfo + 16 * st) = make_int4(n, uniform, 0, 0);
+            *reinterpret_cast<int4*>(smem + C::oInfo + 16 * (j % NCT)) = make_int4(n, uniform, 0, 0);
           }
         }
         ptx::fence_proxy_async_smem();
@@ -655,20 +714,6 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
 template <int QT>
 cudaError_t launch(const CUtensorMap& tm, const AttnParams& prm, cudaStream_t stream) {
   using C = Cfg<QT>;
@@ -685,6 +730,20 @@ cudaError_t launch(const CUtensorMap& tm, const AttnParams& prm, cudaStream_t st
 }
 
 }  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
 
 size_t attention_workspace_bytes(const nvfp4kv_cache&, int) { return 0; }
 
@@ -729,7 +788,7 @@ int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, in
   }
   prm.n_tiles = prm.run_tile0[prm.n_runs];
 
-  PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return NVFP4KV_ERR_CUDA;
   CUtensorMap tm;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(c.heads),

@@ -3,6 +3,8 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "../../include/nvfp4kv.h"
@@ -28,6 +30,9 @@ constexpr size_t kStaticScratchBytes = 64 * 1024;
 cudaError_t static_scratch_address(void** out);
 cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
                             int64_t token_stride, void* workspace, cudaStream_t stream);
+
+// ---- tensor maps (attention.cu): the driver's encoder, looked up once; null if unavailable.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // ---- attention (attention.cu)
 size_t attention_workspace_bytes(const nvfp4kv_cache& c, int q_tokens);

@@ -59,6 +59,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uin
   return ok != 0;
 }
 
+// ---------------------------------------------------------------- clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster arrives; release orders this thread's earlier
+// shared-memory writes before the peers' acquire-waits.
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 32-bit load from the shared memory of CTA `rank` of the cluster, at the offset of the local
+// shared address `addr`.
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t addr, uint32_t rank) {
+  uint32_t remote, v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(rank));
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+  return v;
+}
+
 // ---------------------------------------------------------------- fences
 // Generic-proxy shared-memory writes -> visible to the async proxy (TMA, tensor core).
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -161,6 +184,65 @@ __device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint6
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// A whole 128 x 128 x 128 product as eight K = 16 steps from one elected lane, descriptors
+// advanced in-line (their 14-bit start-address field only; operands lie below 256 KB so the field
+// cannot carry).  The first step accumulates iff `accumulate`, the rest always do.
+//   QK form: A and B K-major, 128B swizzle; step k starts 32 B further inside the 128-byte
+//            atom row, steps 4..7 in the second 64-element half (+16384 B).
+__device__ __forceinline__ void mma_qk8_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t.reg .b32 alo, ahi, blo, bhi, t0, t1;\n\t.reg .b64 da, db;\n\t"
+      "mov.b64 {alo, ahi}, %1;\n\tmov.b64 {blo, bhi}, %2;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "add.s32 t0, alo, 2;\n\tadd.s32 t1, blo, 2;\n\tmov.b64 da, {t0, ahi};\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+      "add.s32 t0, alo, 4;\n\tadd.s32 t1, blo, 4;\n\tmov.b64 da, {t0, ahi};\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+      "add.s32 t0, alo, 6;\n\tadd.s32 t1, blo, 6;\n\tmov.b64 da, {t0, ahi};\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+      "add.s32 t0, alo, 1024;\n\tadd.s32 t1, blo, 1024;\n\tmov.b64 da, {t0, ahi};\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+      "add.s32 t0, alo, 1026;\n\tadd.s32 t1, blo, 1026;\n\tmov.b64 da, {t0, ahi};\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+      "add.s32 t0, alo, 1028;\n\tadd.s32 t1, blo, 1028;\n\tmov.b64 da, {t0, ahi};\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t"
+      "add.s32 t0, alo, 1030;\n\tadd.s32 t1, blo, 1030;\n\tmov.b64 da, {t0, ahi};\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, 1;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+//   PV form: A (P, fp16) in TMEM, 8 columns per K = 16 step; B MN-major with 128B swizzle,
+//            step k 2048 B further (16 rows of 128 B).
+__device__ __forceinline__ void mma_pv8_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t.reg .b32 blo, bhi, t1, ta;\n\t.reg .b64 db;\n\t"
+      "mov.b64 {blo, bhi}, %2;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.s32 ta, %1, 8;\n\tadd.s32 t1, blo, 128;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 16;\n\tadd.s32 t1, blo, 256;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 24;\n\tadd.s32 t1, blo, 384;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 32;\n\tadd.s32 t1, blo, 512;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 40;\n\tadd.s32 t1, blo, 640;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 48;\n\tadd.s32 t1, blo, 768;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 56;\n\tadd.s32 t1, blo, 896;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -378,6 +460,32 @@ __device__ __forceinline__ float add_f16x2_f32(float acc, uint32_t h2) {
       : "+f"(acc)
       : "r"(h2));
   return acc;
+}
+
+// (d0, d1) = (a0, a1) * b + c, one packed fp32 FMA (each lane rounds like fmaf).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %4};\n\t"
+      "mov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
+// 2^x on the FMA pipe, for x <= 2^20: x = n + f with n = round(x) (the 1.5 * 2^23 shift leaves n
+// in the low mantissa bits) and f in [-1/2, 1/2]; 2^f by a cubic fitted to minimum maximum relative
+// error on that interval (Lawson's iteration; max relative error 7.5e-5, below half an fp16 ulp);
+// n is added to the exponent field.  Inputs below -125 return 2^-125 * 2^f (far below fp16 range).
+constexpr float kExp2C0 = 0.99992811f, kExp2C1 = 0.69326099f, kExp2C2 = 0.24261054f,
+                kExp2C3 = 0.05517132f;
+__device__ __forceinline__ float ex2_poly3(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ float ex2(float x) {

@@ -3,21 +3,28 @@
 // Method: "LongLive-2.0" reading note (yingwang.github.io), "The inference infrastructure"
 // (K and V re-quantised to NVFP4 at frame-chunk granularity) and "The NVFP4 quantization
 // format" (FP32 scale, E4M3 scale per 16 elements, E2M1 elements); constants 16 / 448 / 6
-// from the paper page, section 2.2 "NVFP4 Training".  The per-(chunk, head) FP32 scale
-// needs the chunk maximum before any element can be encoded, so the work is two
-// memory-bound passes over the bf16 input:
-//   pass 1 (amax_kernel)     every CTA reduces a token range of one (b, h, tensor) to
-//                            max|x| and writes it to a workspace slot (no atomics, no
-//                            zero-fill, deterministic);
-//   pass 2 (quantize_kernel) every CTA folds the partial maxima of its (b, h, tensor) into
-//                            g, then encodes its token range: two lanes per 16-element
-//                            block, 16-byte loads, a shuffle for the block maximum, hardware
-//                            RNE/satfinite conversions to E4M3 and E2M1, 4-byte code stores
-//                            that are contiguous across the warp.
-// The second pass re-reads its input right after the first, from L2 for chunks that fit.
-// Every fp32 step uses an explicitly rounded intrinsic (no contraction, no flush to zero),
-// so the codes are bit-identical to the fp32 definition of the method.
+// from the paper page, section 2.2 "NVFP4 Training".  The per-(chunk, head) FP32 scale needs
+// the chunk maximum before any element can be encoded.  Two paths, the same arithmetic:
+//   single pass (quantize_cluster_kernel), when one cluster per (b, h, tensor) fits the GPU in
+//       one wave: the cluster's CTAs TMA their token rows into shared memory, reduce max|x|,
+//       exchange the maxima through distributed shared memory, and encode from shared memory
+//       (the input crosses HBM once);
+//   two passes otherwise:
+//       amax_kernel      every CTA reduces 128 tokens of one (b, h, tensor) to max|x| and writes
+//                        it to a workspace slot (no atomics, no zero-fill, deterministic);
+//       quantize_kernel  launched as a programmatic dependent of the amax grid: every CTA loads
+//                        its 128 rows (from L2, where the first pass just read them), then waits
+//                        for the amax grid, folds the partial maxima into g and encodes.
+// Encoding: two lanes per 16-element block, 16-byte loads, a shuffle for the block maximum,
+// hardware RNE/satfinite conversions to E4M3 and E2M1, 4-byte code stores contiguous across the
+// warp.  Every fp32 step is an explicitly rounded intrinsic (no contraction, no flush to zero),
+// and the two shortcuts (a hoisted reciprocal with an exact FMA correction for the block-scale
+// quotient, a per-code reciprocal table) reproduce the correctly rounded operations, so the codes
+// are bit-identical to the fp32 definition of the method.
+#include <algorithm>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -27,7 +34,11 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kTargetCtas = 148 * 4;  // four CTAs per SM in flight on a B200
+// Two-pass path: a CTA owns kPartTokens tokens of one (b, h, tensor); 16 threads read a 256-byte
+// token row, so the CTA covers 16 rows per pass and issues all kPasses loads of every thread
+// before it uses any (one memory latency per CTA).
+constexpr int kPasses = 8;
+constexpr int kPartTokens = (kThreads / 16) * kPasses;  // 128
 
 struct QuantArgs {
   const uint16_t* x[2];  // K, V (bf16 bits)
@@ -37,7 +48,7 @@ struct QuantArgs {
   uint32_t* partial;  // [2][B*H][parts], bf16 bit pattern of a partial max|x|
   int64_t token_stride;
   int64_t T;  // tokens per (b, h) in the cache
-  int B, H, L, C, slot, parts, tokens_per_part;
+  int B, H, L, C, slot, parts;
 };
 
 __device__ __forceinline__ uint4 ld_row16(const uint16_t* p) {
@@ -55,26 +66,93 @@ __device__ __forceinline__ uint32_t absmax_bits(uint4 w) {
   return m;
 }
 
+// Per-CTA encoder state for one (chunk, head, tensor).  The block-scale quotient a_b / (6 g) is
+// the correctly rounded fp32 quotient: with y = RN(1 / d) and q = RN(a_b * y), the residual
+// r = a_b - q d is exact in one FMA and RN(q + r y) = RN(a_b / d) (Markstein's correction
+// theorem), valid while nothing underflows, i.e. for normal d and y and a_b >= 2^-100; smaller
+// block maxima take the IEEE division.  rtab[c] = RN(1 / RN(s_c * g)) for every E4M3 code c of the
+// block scale, or 0 where the block's codes are all zero (s_c = 0, or the reciprocal overflows).
+struct Encoder {
+  float g, d, y;
+  bool fast;
+};
+
+__device__ __forceinline__ Encoder make_encoder(float g, float* rtab, int tid, int nthreads) {
+  Encoder e;
+  e.g = g;
+  e.d = __fmul_rn(6.0f, g);
+  e.y = g != 0.0f ? __frcp_rn(e.d) : 0.0f;
+  e.fast = g != 0.0f && e.d >= 0x1p-126f && e.y >= 0x1p-126f && e.y < 0x1p127f;
+  for (int c = tid; c < 128; c += nthreads) {
+    const float s = ptx::e4m3_to_f32(static_cast<uint32_t>(c));
+    float r = 0.0f;
+    if (s != 0.0f && c != 0x7F) {
+      r = __frcp_rn(__fmul_rn(s, g));
+      if (r == __int_as_float(0x7F800000)) r = 0.0f;
+    }
+    rtab[c] = r;
+  }
+  return e;
+}
+
+// Encodes this lane's 8 elements of a 16-element block (its partner lane xor 1 holds the other 8)
+// and stores the 4 code bytes and, from the even lane, the scale byte.
+__device__ __forceinline__ void encode_store(uint4 w, const Encoder& e, const float* rtab, bool valid,
+                                             uint8_t* code_dst, uint8_t* scale_dst, int lane) {
+  uint32_t mb = absmax_bits(w);
+  mb = max(mb & 0xFFFFu, mb >> 16);
+  mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 1));
+  const float ab = __uint_as_float(mb << 16);
+  uint32_t s_code = 0;
+  if (ab != 0.0f && e.g != 0.0f) {
+    float q;
+    if (e.fast && ab >= 0x1p-100f) {
+      q = __fmul_rn(ab, e.y);
+      const float r = __fmaf_rn(-q, e.d, ab);
+      q = __fmaf_rn(r, e.y, q);
+    } else {
+      q = __fdiv_rn(ab, e.d);
+    }
+    s_code = ptx::f32_to_e4m3(q);
+  }
+  const float r = rtab[s_code & 0x7F];
+  uint32_t qc = 0;
+  if (r != 0.0f) {
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      y[2 * i] = __fmul_rn(__uint_as_float(wv[i] << 16), r);
+      y[2 * i + 1] = __fmul_rn(__uint_as_float(wv[i] & 0xFFFF0000u), r);
+    }
+    qc = ptx::f32x8_to_e2m1x8(y);
+  }
+  if (valid) {
+    *reinterpret_cast<uint32_t*>(code_dst) = qc;
+    if ((lane & 1) == 0) *scale_dst = static_cast<uint8_t>(s_code);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads) amax_kernel(const __grid_constant__ QuantArgs a) {
   const int part = blockIdx.x, bh = blockIdx.y, tensor = blockIdx.z;
   const int b = bh / a.H, h = bh % a.H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t_begin = part * a.tokens_per_part;
-  const int t_end = min(a.L, t_begin + a.tokens_per_part);
+  // the dependent encode grid may start loading its rows now; it waits for this grid's results
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int t_begin = part * kPartTokens;
+  const int t_end = min(a.L, t_begin + kPartTokens);
+  const int sub = threadIdx.x >> 4;
   const uint16_t* x = a.x[tensor] + static_cast<int64_t>(b) * a.L * a.token_stride +
-                      static_cast<int64_t>(h) * kHeadDim + (lane & 15) * 8;
-  uint32_t acc = 0;
-  constexpr int kUnroll = 4;
-  for (int t0 = t_begin + 2 * warp; t0 < t_end; t0 += 2 * kWarps * kUnroll) {
-    uint4 w[kUnroll];
+                      static_cast<int64_t>(h) * kHeadDim + (threadIdx.x & 15) * 8;
+  uint4 w[kPasses];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int t = t0 + 2 * kWarps * u + (lane >> 4);
-      w[u] = (t < t_end) ? ld_row16(x + t * a.token_stride) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) acc = __vmaxu2(acc, absmax_bits(w[u]));
+  for (int u = 0; u < kPasses; ++u) {
+    const int t = t_begin + u * (kThreads / 16) + sub;
+    w[u] = t < t_end ? ld_row16(x + static_cast<int64_t>(t) * a.token_stride) : make_uint4(0, 0, 0, 0);
   }
+  uint32_t acc = 0;
+#pragma unroll
+  for (int u = 0; u < kPasses; ++u) acc = __vmaxu2(acc, absmax_bits(w[u]));
   uint32_t m = max(acc & 0xFFFFu, acc >> 16);
   m = __reduce_max_sync(0xFFFFFFFFu, m);
   __shared__ uint32_t red[kWarps];
@@ -92,6 +170,20 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const __grid_constan
   const int part = blockIdx.x, bh = blockIdx.y, tensor = blockIdx.z;
   const int b = bh / a.H, h = bh % a.H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t_begin = part * kPartTokens;
+  const int t_end = min(a.L, t_begin + kPartTokens);
+  const int sub = threadIdx.x >> 4;
+  const uint16_t* x = a.x[tensor] + static_cast<int64_t>(b) * a.L * a.token_stride +
+                      static_cast<int64_t>(h) * kHeadDim + (threadIdx.x & 15) * 8;
+  // The rows do not depend on the amax grid: they are loaded (mostly from L2, where that grid
+  // just read them) before waiting for its partial maxima.
+  uint4 w[kPasses];
+#pragma unroll
+  for (int u = 0; u < kPasses; ++u) {
+    const int t = t_begin + u * (kThreads / 16) + sub;
+    w[u] = t < t_end ? ld_row16(x + static_cast<int64_t>(t) * a.token_stride) : make_uint4(0, 0, 0, 0);
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // FP32 scale of this (chunk, head, tensor): g = max|x| / (448 * 6).
   __shared__ float s_g;
@@ -107,63 +199,155 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const __grid_constan
       if (part == 0) a.gscale[tensor][static_cast<int64_t>(bh) * a.C + a.slot] = g;
     }
   }
+  __shared__ float rtab[128];
   __syncthreads();
-  const float g = s_g;
-  const float denom = __fmul_rn(6.0f, g);
+  const Encoder enc = make_encoder(s_g, rtab, threadIdx.x, kThreads);
+  __syncthreads();
 
-  const int t_begin = part * a.tokens_per_part;
-  const int t_end = min(a.L, t_begin + a.tokens_per_part);
-  const uint16_t* x = a.x[tensor] + static_cast<int64_t>(b) * a.L * a.token_stride +
-                      static_cast<int64_t>(h) * kHeadDim + (lane & 15) * 8;
   const int64_t row0 = static_cast<int64_t>(bh) * a.T + static_cast<int64_t>(a.slot) * a.L;
   uint8_t* codes = a.codes[tensor] + row0 * kCodeBytes + (lane & 15) * 4;
   uint8_t* scales = a.scales[tensor] + row0 * kScaleBytes + ((lane & 15) >> 1);
-
-  // Warp-uniform trip count: lanes 0-15 take the even token of a pair, 16-31 the odd one.
-  for (int t0 = t_begin + 2 * warp; t0 < t_end; t0 += 2 * kWarps) {
-    const int t = t0 + (lane >> 4);
-    const bool valid = t < t_end;
-    const uint4 w = valid ? ld_row16(x + t * a.token_stride) : make_uint4(0, 0, 0, 0);
-    uint32_t mb = absmax_bits(w);
-    mb = max(mb & 0xFFFFu, mb >> 16);
-    mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 1));  // the two lanes of one 16-element block
-    const float ab = __uint_as_float(mb << 16);
-
-    uint32_t s_code = 0;
-    if (ab != 0.0f && g != 0.0f) s_code = ptx::f32_to_e4m3(__fdiv_rn(ab, denom));
-    const float s = ptx::e4m3_to_f32(s_code);
-    uint32_t q = 0;
-    if (s != 0.0f) {
-      const float r = __frcp_rn(__fmul_rn(s, g));
-      if (r != __int_as_float(0x7F800000)) {  // 1/(s*g) overflowed: the block stays zero
-        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-        float y[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          y[2 * i] = __fmul_rn(__uint_as_float(wv[i] << 16), r);
-          y[2 * i + 1] = __fmul_rn(__uint_as_float(wv[i] & 0xFFFF0000u), r);
-        }
-        q = ptx::f32x8_to_e2m1x8(y);
+  for (int u = 0; u < kPasses; ++u) {
+    const int t = t_begin + u * (kThreads / 16) + sub;
+    encode_store(w[u], enc, rtab, t < t_end, codes + static_cast<int64_t>(t) * kCodeBytes,
+                 scales + static_cast<int64_t>(t) * kScaleBytes, lane);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Single-pass path: one thread-block cluster per (b, h, tensor).  The cluster's CTAs split the
+// chunk's tokens; each CTA brings its rows into shared memory with TMA (the input is read from
+// HBM once), reduces its max|x|, and the CTAs exchange their maxima through distributed shared
+// memory before every CTA encodes its rows from shared memory.
+constexpr int kBoxTokens = 16;          // tokens per TMA box (16 x 256 B)
+constexpr int kMaxCtaTokens = 448;      // 112 KB of bf16 rows: two CTAs per SM
+constexpr int kMaxCluster = 16;
+#ifndef NVFP4KV_QC_THREADS
+#define NVFP4KV_QC_THREADS 512
+#endif
+constexpr int kCThreads = NVFP4KV_QC_THREADS;
+constexpr int kCWarps = kCThreads / 32;
+
+struct ClusterArgs {
+  uint8_t* codes[2];
+  uint8_t* scales[2];
+  float* gscale[2];
+  uint32_t* status;
+  int64_t T;  // tokens per (b, h) in the cache
+  int H, L, C, slot, cta_tokens;
+};
+
+__global__ void __launch_bounds__(kCThreads)
+    quantize_cluster_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                            const __grid_constant__ ClusterArgs a) {
+  extern __shared__ __align__(128) uint8_t qsm[];
+  __shared__ __align__(8) uint64_t full_bar;
+  __shared__ uint32_t red[kCWarps];
+  __shared__ uint32_t cta_max;
+  __shared__ float s_g;
+  __shared__ float rtab[128];
+  const uint32_t rank = ptx::cluster_ctarank();
+  const int bh = blockIdx.y, tensor = blockIdx.z;
+  const int b = bh / a.H, h = bh % a.H;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = static_cast<int>(rank) * a.cta_tokens;
+  const int n = max(0, min(a.L - t0, a.cta_tokens));
+  const int nbox = (n + kBoxTokens - 1) / kBoxTokens;
+  const uint32_t bar = ptx::smem_u32(&full_bar);
+  const uint32_t xs = ptx::smem_u32(qsm);
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar, 1);
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && nbox > 0) {
+    const CUtensorMap* tm = tensor == 0 ? &tm_k : &tm_v;
+    ptx::mbar_arrive_expect_tx(bar, nbox * kBoxTokens * kHeadDim * 2);
+    for (int i = 0; i < nbox; ++i)
+      ptx::tma_load_4d(xs + i * kBoxTokens * kHeadDim * 2, tm, 0, h, t0 + i * kBoxTokens, b, bar);
+  }
+  bool ok = true;
+  if (nbox > 0) {
+    uint64_t w0 = 0;
+    int it = 0;
+    while (!ptx::mbar_try_wait(bar, 0)) {
+      const uint64_t now = ptx::globaltimer_ns();
+      if (it++ == 0) w0 = now;
+      if (now - w0 > kWaitLimitNs) {
+        ok = false;
+        break;
       }
     }
-    if (valid) {
-      *reinterpret_cast<uint32_t*>(codes + static_cast<int64_t>(t) * kCodeBytes) = q;
-      if ((lane & 1) == 0) scales[static_cast<int64_t>(t) * kScaleBytes] = static_cast<uint8_t>(s_code);
+  }
+  ok = __syncthreads_and(ok) != 0;
+  if (!ok && threadIdx.x == 0) atomicOr(a.status, kStatusTimeout);
+
+  // max|x| over this CTA's rows (bf16 magnitudes compare as integers)
+  const uint16_t* rows = reinterpret_cast<const uint16_t*>(qsm) + (lane & 15) * 8;
+  uint32_t acc = 0;
+  if (ok)
+    for (int t = 2 * warp + (lane >> 4); t < n; t += 2 * kCWarps)
+      acc = __vmaxu2(acc, absmax_bits(*reinterpret_cast<const uint4*>(rows + t * kHeadDim)));
+  uint32_t m = max(acc & 0xFFFFu, acc >> 16);
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t r = 0;
+#pragma unroll
+    for (int i = 0; i < kCWarps; ++i) r = max(r, red[i]);
+    cta_max = r;
+  }
+  // Exchange the maxima: every CTA's cta_max is written before the barrier; warp 0 then reads
+  // all of them.  The second barrier's wait (at the end) keeps every CTA's shared memory alive
+  // until all peers have read it.
+  ptx::cluster_arrive_release();
+  ptx::cluster_wait_acquire();
+  if (warp == 0) {
+    const uint32_t ncta = gridDim.x;
+    uint32_t r = lane < static_cast<int>(ncta) ? ptx::ld_shared_cluster_u32(ptx::smem_u32(&cta_max), lane) : 0u;
+    r = __reduce_max_sync(0xFFFFFFFFu, r);
+    if (lane == 0) {
+      const float A = __uint_as_float(r << 16);
+      s_g = (A == 0.0f) ? 0.0f : __fdiv_rn(A, 2688.0f);
     }
   }
+  ptx::cluster_arrive_release();
+  __syncthreads();
+  const float g = s_g;
+  if (ok && rank == 0 && threadIdx.x == 0) a.gscale[tensor][static_cast<int64_t>(bh) * a.C + a.slot] = g;
+  const Encoder enc = make_encoder(g, rtab, threadIdx.x, kCThreads);
+  __syncthreads();
+  const int64_t row0 = static_cast<int64_t>(bh) * a.T + static_cast<int64_t>(a.slot) * a.L + t0;
+  uint8_t* codes = a.codes[tensor] + row0 * kCodeBytes + (lane & 15) * 4;
+  uint8_t* scales = a.scales[tensor] + row0 * kScaleBytes + ((lane & 15) >> 1);
+  if (ok) {
+    // warp-uniform trip count; two independent token pairs per pass (lanes 0-15 take the even
+    // token of a pair, 16-31 the odd one)
+    for (int tp = 4 * warp; tp < n; tp += 4 * kCWarps) {
+      const int ta = tp + (lane >> 4), tb = ta + 2;
+      const uint4 wa = ta < n ? *reinterpret_cast<const uint4*>(rows + ta * kHeadDim) : make_uint4(0, 0, 0, 0);
+      const uint4 wb = tb < n ? *reinterpret_cast<const uint4*>(rows + tb * kHeadDim) : make_uint4(0, 0, 0, 0);
+      encode_store(wa, enc, rtab, ta < n, codes + static_cast<int64_t>(ta) * kCodeBytes,
+                   scales + static_cast<int64_t>(ta) * kScaleBytes, lane);
+      encode_store(wb, enc, rtab, tb < n, codes + static_cast<int64_t>(tb) * kCodeBytes,
+                   scales + static_cast<int64_t>(tb) * kScaleBytes, lane);
+    }
+  } else if (nbox > 0 && threadIdx.x == 0) {
+    // the copies were issued: let them land before the CTA's shared memory goes away
+    uint64_t w0 = ptx::globaltimer_ns();
+    while (!ptx::mbar_try_wait(bar, 0))
+      if (ptx::globaltimer_ns() - w0 > kWaitLimitNs) break;
+  }
+  ptx::cluster_wait_acquire();
 }
 
 }  // namespace
 
-int quantize_parts(int batch, int heads, int chunk_tokens) {
-  const int units = 2 * batch * heads;
-  int parts = (kTargetCtas + units - 1) / units;
-  const int max_parts = (chunk_tokens + 15) / 16;  // at least 16 tokens per CTA
-  if (parts > max_parts) parts = max_parts;
-  if (parts < 1) parts = 1;
-  int tpp = (chunk_tokens + parts - 1) / parts;
-  tpp = (tpp + 1) & ~1;
-  return (chunk_tokens + tpp - 1) / tpp;
+int quantize_parts(int, int, int chunk_tokens) {
+  return chunk_tokens > 0 ? (chunk_tokens + kPartTokens - 1) / kPartTokens : 1;
 }
 
 size_t quantize_workspace_bytes(int batch, int heads, int chunk_tokens) {
@@ -171,8 +355,114 @@ size_t quantize_workspace_bytes(int batch, int heads, int chunk_tokens) {
          sizeof(uint32_t);
 }
 
+namespace {
+
+// Cluster size for the single-pass path, or 0 when the chunk does not fit it: about two CTAs
+// per SM over the whole grid, at least 16 tokens and at most kMaxCtaTokens rows per CTA.
+int cluster_size(int units, int L) {
+  int cl = std::max(1, std::min(kMaxCluster, (2 * 148) / std::max(1, units)));
+  cl = std::min(cl, std::max(1, L / 16));
+  while (cl < kMaxCluster && (L + cl - 1) / cl > kMaxCtaTokens) ++cl;
+  return (L + cl - 1) / cl > kMaxCtaTokens ? 0 : cl;
+}
+
+cudaError_t launch_cluster(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
+                           int64_t token_stride, int cl, cudaStream_t stream, bool* launched) {
+  *launched = false;
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return cudaSuccess;
+  ClusterArgs a;
+  a.codes[0] = c.k_codes;
+  a.codes[1] = c.v_codes;
+  a.scales[0] = c.k_scales;
+  a.scales[1] = c.v_scales;
+  a.gscale[0] = c.k_gscale;
+  a.gscale[1] = c.v_gscale;
+  a.status = c.status;
+  a.T = static_cast<int64_t>(c.capacity_chunks) * c.chunk_tokens;
+  a.H = c.heads;
+  a.L = c.chunk_tokens;
+  a.C = c.capacity_chunks;
+  a.slot = slot;
+  a.cta_tokens = ((c.chunk_tokens + cl - 1) / cl + kBoxTokens - 1) / kBoxTokens * kBoxTokens;
+  CUtensorMap tm[2];
+  const uint16_t* src[2] = {k, v};
+  for (int i = 0; i < 2; ++i) {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(c.heads),
+                                static_cast<cuuint64_t>(c.chunk_tokens), static_cast<cuuint64_t>(c.batch)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHeadDim) * 2,
+                                   static_cast<cuuint64_t>(token_stride) * 2,
+                                   static_cast<cuuint64_t>(c.chunk_tokens) * token_stride * 2};
+    const cuuint32_t box[4] = {kHeadDim, 1, kBoxTokens, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (encode(&tm[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(src[i]), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaSuccess;  // not expressible as a tensor map: the two-pass path takes it
+  }
+  const size_t smem = static_cast<size_t>(a.cta_tokens) * kHeadDim * 2;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(quantize_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kMaxCtaTokens * kHeadDim * 2);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(quantize_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  });
+  if (attr_err != cudaSuccess) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cl, c.batch * c.heads, 2);
+  cfg.blockDim = dim3(kCThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // How many clusters of this shape can be resident at once, asked once per (device, shape).  The
+  // path is only worth taking when every (b, h, tensor) gets its cluster in the first wave: a
+  // second wave would wait for the first to finish its whole load-reduce-encode sequence.
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, size_t>, int> active;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaSuccess;
+  int max_active = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_tuple(dev, cl, smem);
+    auto it = active.find(key);
+    if (it == active.end()) {
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, quantize_cluster_kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        clusters = 0;
+      }
+      it = active.emplace(key, clusters).first;
+    }
+    max_active = it->second;
+  }
+  if (max_active < 2 * c.batch * c.heads) return cudaSuccess;  // the two-pass path takes it
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_cluster_kernel, tm[0], tm[1], a);
+  *launched = e == cudaSuccess;
+  return e;
+}
+
+}  // namespace
+
 cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
                             int64_t token_stride, void* workspace, cudaStream_t stream) {
+#ifndef NVFP4KV_QUANT_CLUSTER
+#define NVFP4KV_QUANT_CLUSTER 1
+#endif
+  const int cl = NVFP4KV_QUANT_CLUSTER ? cluster_size(2 * c.batch * c.heads, c.chunk_tokens) : 0;
+  if (cl > 0) {
+    bool launched = false;
+    const cudaError_t e = launch_cluster(c, slot, k, v, token_stride, cl, stream, &launched);
+    if (launched || e != cudaSuccess) return e;
+  }
   QuantArgs a;
   a.x[0] = k;
   a.x[1] = v;
@@ -191,12 +481,22 @@ cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k,
   a.C = c.capacity_chunks;
   a.slot = slot;
   a.parts = quantize_parts(c.batch, c.heads, c.chunk_tokens);
-  int tpp = (c.chunk_tokens + a.parts - 1) / a.parts;
-  a.tokens_per_part = (tpp + 1) & ~1;
   const dim3 grid(a.parts, c.batch * c.heads, 2);
   amax_kernel<<<grid, kThreads, 0, stream>>>(a);
-  quantize_kernel<<<grid, kThreads, 0, stream>>>(a);
-  return cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // The encode grid is a programmatic dependent of the amax grid: it launches while the amax grid
+  // drains and waits (griddepcontrol.wait) only before it reads the partial maxima.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_kernel, a);
 }
 
 // ---------------------------------------------------------------------------------------

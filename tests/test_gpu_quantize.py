@@ -57,14 +57,23 @@ def test_quantize_matches_oracle_bit_for_bit(key, slots):
     assert cache.read_status() == 0
 
 
+# Chunks of up to 16 x 448 tokens per (b, h) are quantised by one thread-block cluster in a single
+# pass; longer ones by the two-pass kernels.  Every special chunk runs through both.
+TWO_PASS_TOKENS = 7200
+
+
+@pytest.mark.parametrize("path", ["cluster", "two_pass"])
 @pytest.mark.parametrize("name", ["fixed0", "fixed-20", "fixed17", "fixed-100", "ties0", "ties-9",
                                   "underflow", "tiny_scale"])
-def test_special_chunks_match_oracle(name):
+def test_special_chunks_match_oracle(name, path):
     chunk = {"fixed0": lambda: sc.fixed_point_chunk(0), "fixed-20": lambda: sc.fixed_point_chunk(-20),
              "fixed17": lambda: sc.fixed_point_chunk(17), "fixed-100": lambda: sc.fixed_point_chunk(-100),
              "ties0": lambda: sc.tie_chunk(0), "ties-9": lambda: sc.tie_chunk(-9),
              "underflow": sc.underflow_chunk, "tiny_scale": sc.tiny_scale_chunk}[name]()
     chunk = sc.pad_tokens(chunk)
+    if path == "two_pass":
+        reps = -(-TWO_PASS_TOKENS // chunk.shape[1])
+        chunk = np.ascontiguousarray(np.tile(chunk, (1, reps, 1, 1)))
     L = chunk.shape[1]
     cache = KVCache(1, 1, L, 2)
     ocache = oracle.Cache(1, 1, 128, L, 2)
@@ -74,6 +83,13 @@ def test_special_chunks_match_oracle(name):
     assert_cache_equal(cache, ocache, [1])
     # the slot not written stays untouched
     assert int(cache.k_codes[:, :, :L].abs().sum()) == 0
+
+
+def test_long_chunk_two_pass_path_matches_oracle():
+    w = dataclasses.replace(synthetic.WORKLOADS["tiny"], heads=2, chunk_tokens=TWO_PASS_TOKENS + 8, capacity=2)
+    cache, ocache = make_caches(w, [1])
+    assert_cache_equal(cache, ocache, [1])
+    assert cache.read_status() == 0
 
 
 def test_token_stride_fused_qkv_layout():
