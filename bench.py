@@ -301,6 +301,7 @@ def main():
         dist.barrier()
 
     attn_flops, attn_bytes, quant_bytes = work(w)
+    q_launches = sets[0]["cache"].quantize_launches()
     ms_per_step = elapsed_ms / args.steps
     step_flops = attn_flops * w.attn_calls
     value = step_flops * world / (ms_per_step * 1e-3) / 1e12
@@ -331,13 +332,15 @@ def main():
                          "algorithmic_flops_per_launch": attn_flops,
                          "algorithmic_bytes_per_launch": attn_bytes,
                          "launch_us": t_attn * 1e3},
-            "quantize": {"bound": "hbm", "kernels": "amax_kernel + quantize_kernel",
+            "quantize": {"bound": "hbm",
+                         "kernels": ("quantize_cluster_kernel" if q_launches == 1
+                                     else "amax_kernel + quantize_kernel"),
                          "achieved": quant_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": quant_gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_call": quant_bytes,
                          "call_us": t_quant * 1e3, "peak_source": f"{src} HBM copy"},
             "e2e": {"value": step_flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": args.steps * (2 + w.attn_calls),
+            "gpu_launches": args.steps * (q_launches + w.attn_calls),
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -99,9 +99,11 @@ size_t nvfp4kv_workspace_bytes(const nvfp4kv_cache* cache, int32_t q_tokens);
  *   workspace       device scratch of at least nvfp4kv_workspace_bytes() bytes, 16-byte
  *                   aligned; its contents on entry do not matter
  * Writes codes, scales and the FP32 scales of slot `chunk_slot` for every (b, h); nothing
- * else in the cache is touched.  Bit-for-bit deterministic.
+ * else in the cache is touched.  Bit-for-bit deterministic, and the same bits whichever of the
+ * two kernel paths runs (nvfp4kv_quantize_launches tells which).
  * Errors: NVFP4KV_ERR_INVALID_ARG (null, misaligned, slot out of range, bad stride),
- * NVFP4KV_ERR_UNSUPPORTED, NVFP4KV_ERR_WORKSPACE, NVFP4KV_ERR_CUDA (launch failed). */
+ * NVFP4KV_ERR_UNSUPPORTED, NVFP4KV_ERR_WORKSPACE, NVFP4KV_ERR_CUDA (launch failed); a device
+ * wait that ran out sets the status bit of NVFP4KV_ERR_DEVICE_TIMEOUT. */
 int nvfp4_kv_quantize(const nvfp4kv_cache* cache, int32_t chunk_slot, const void* k_bf16,
                       const void* v_bf16, int64_t token_stride, void* workspace,
                       size_t workspace_bytes, void* cuda_stream);
@@ -113,9 +115,9 @@ int nvfp4_kv_quantize(const nvfp4kv_cache* cache, int32_t chunk_slot, const void
  * Same arguments, results and errors as nvfp4_kv_quantize, except that the amax partials
  * live in a fixed 64 KiB device array inside the library, which every GPU that loads the
  * library keeps until the process exits.  It calls no cudaMalloc or cudaFree.
- *  - Caches needing more partials than fit (2 * batch * heads * parts * 4 bytes, about
- *    2 * batch * heads * 4 bytes for large batch * heads) are rejected with
- *    NVFP4KV_ERR_WORKSPACE before anything is launched; use nvfp4_kv_quantize for them.
+ *  - Caches needing more partials than fit (2 * batch * heads * ceil(chunk_tokens / 128) * 4
+ *    bytes) are rejected with NVFP4KV_ERR_WORKSPACE before anything is launched; use
+ *    nvfp4_kv_quantize for them.
  *  - The first call on each device looks up the array's device address (with that device
  *    current), which may load the library's GPU code: make that first call before any
  *    stream capture.
@@ -158,6 +160,13 @@ int nvfp4_kv_dequantize(const nvfp4kv_cache* cache, int32_t which, int32_t first
  * format definition over whole ranges of inputs. */
 int nvfp4kv_debug_encode(const float* x, int64_t n, uint8_t* e2m1_codes, uint8_t* e4m3_codes,
                          void* cuda_stream);
+
+/* Kernels that nvfp4_kv_quantize (and its static-scratch variant) launch per call for this cache
+ * shape on the current device: 1 when every (batch, head, tensor) gets one thread-block cluster
+ * in a single wave (single pass: the input crosses HBM once), 2 otherwise (an amax pass and an
+ * encode pass).  Both paths write the same bits.  A library diagnostic with no counterpart in
+ * the pages; a negative result is minus an nvfp4kv_status code (invalid cache, no sm_100 device). */
+int nvfp4kv_quantize_launches(const nvfp4kv_cache* cache);
 
 /* Wait for `cuda_stream`, then read the cache's device status word into *out and clear it.
  * *out == 0 means no device-side error since the last read; otherwise it holds OR-ed

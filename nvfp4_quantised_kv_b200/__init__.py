@@ -50,6 +50,7 @@ SIGNATURES = {
                                           _vp, _i32, _vp, _sz, _vp]),
     "nvfp4_kv_dequantize": (ctypes.c_int, [_CP, _i32, _i32, _i32, _vp, _vp]),
     "nvfp4kv_debug_encode": (ctypes.c_int, [_vp, _i64, _vp, _vp, _vp]),
+    "nvfp4kv_quantize_launches": (ctypes.c_int, [_CP]),
     "nvfp4kv_read_status": (ctypes.c_int, [_CP, _vp, ctypes.POINTER(ctypes.c_uint32)]),
     "nvfp4kv_strerror": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -164,6 +165,13 @@ class KVCache:
         _check(lib().nvfp4_kv_quantize(ctypes.byref(self.desc), slot, k.data_ptr(), v.data_ptr(), ks,
                                        self._ws.data_ptr(), self._ws.numel(), _stream_handle(stream)),
                "nvfp4_kv_quantize")
+
+    def quantize_launches(self) -> int:
+        """Kernels one ``quantize`` call launches for this cache on the current device (1 or 2)."""
+        n = lib().nvfp4kv_quantize_launches(ctypes.byref(self.desc))
+        if n < 0:
+            raise NvFp4KvError(-n, "nvfp4kv_quantize_launches")
+        return n
 
     def attention(self, q, q_chunk: int, n_sink: int, window: int, softmax_scale: float = 0.0,
                   out=None, out_dtype=None, stream=None):

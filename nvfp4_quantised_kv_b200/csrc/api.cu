@@ -158,6 +158,14 @@ int nvfp4kv_debug_encode(const float* x, int64_t n, uint8_t* e2m1_codes, uint8_t
   return e == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 
+int nvfp4kv_quantize_launches(const nvfp4kv_cache* cache) {
+  int rc = check_cache(cache);
+  if (rc != NVFP4KV_OK) return -rc;
+  rc = check_device();
+  if (rc != NVFP4KV_OK) return -rc;
+  return quantize_launches(*cache);
+}
+
 int nvfp4kv_read_status(const nvfp4kv_cache* cache, void* cuda_stream, uint32_t* out) {
   if (!cache || !cache->status || !out) return NVFP4KV_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);

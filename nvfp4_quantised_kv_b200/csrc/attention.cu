@@ -32,7 +32,9 @@
 
 #include <algorithm>
 #include <cmath>
+#include <functional>
 #include <mutex>
+#include <queue>
 #include <vector>
 
 #include "internal.h"
@@ -57,10 +59,6 @@ constexpr int MAX_RUNS = 4;
 #define NVFP4KV_EXP2_EMUL 0
 #endif
 constexpr int kExp2Emul = NVFP4KV_EXP2_EMUL;  // 0: every exponent on the MUFU
-#ifndef NVFP4KV_TURNS
-#define NVFP4KV_TURNS 0
-#endif
-constexpr bool kTurns = NVFP4KV_TURNS != 0;  // the two softmax warpgroups take turns
 
 template <int QT>
 struct Cfg {
@@ -70,7 +68,7 @@ struct Cfg {
   static constexpr int kDequantWarp0 = kSoftmaxWarps + 2;
   static constexpr int kDequantWarps = 6;  // 2 in the producer/MMA warpgroup + one full warpgroup
   static constexpr int kDequantThreads = 32 * kDequantWarps;
-  static_assert(kDequantThreads == 192, "dequant_tile deals blocks to 192 threads");
+  static_assert(kDequantThreads % 64 == 0, "dequant_tile deals blocks to a multiple of 64 threads");
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 2 + kDequantWarps);  // whole warpgroups
   static constexpr uint32_t kTmemCols = QT == 1 ? 256 : 512;
   // shared memory map (bytes from a 1024-aligned base)
@@ -99,8 +97,7 @@ struct Cfg {
   static constexpr int bPFull = bSFull + QT;
   static constexpr int bODone = bPFull + QT;
   static constexpr int bDrain = bODone + QT;
-  static constexpr int bTok = bDrain + 1;  // softmax turn: [0] tile 0 -> tile 1, [1] tile 1 -> tile 0
-  static constexpr int kNumBars = bTok + 2;
+  static constexpr int kNumBars = bDrain + 1;
   static constexpr int oMisc = oBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag
   static constexpr int kSmemBytes = oMisc + 16 + 1024;  // + slack for 1024-B alignment
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -124,6 +121,10 @@ struct AttnParams {
   int run_tile0[MAX_RUNS + 1];
   int n_tiles;
   float scale_log2;  // softmax scale * log2(e)
+  // Work list: every (b, h) has n_qt query tiles of 128 rows; the first pp + 1 (for (b, h) <
+  // pr) or pp of its tile pairs go to two-tile CTAs, the rest of its tiles to one-tile CTAs.
+  // CTAs [0, n_pair_ctas) take pairs, the others single tiles.
+  int n_qt, pp, pr, n_pair_ctas;
 };
 
 // ------------------------------------------------------------------ waits
@@ -205,16 +206,17 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
 
 // Dequantise one packed tile (codes + E4M3 scales of BN keys) into a 128B-swizzled [key][d]
 // operand tile of fp16 values, code * scale (exact: <= 6 significant bits, 2^-10 .. 2688).
-// Thread dt of NT = 192 owns the 16-element block blk = dt % 8 of keys dt / 8 + 24 * it: 192 is a
-// multiple of 8 (the block, the swizzle phase key % 8 and the store order are fixed per thread)
-// and of 24 rows of the operand tile (every address is a per-thread base plus a constant).  All
+// Thread dt of NT owns the 16-element block blk = dt % 8 of keys dt / 8 + (NT / 8) * it: NT / 8 is
+// a multiple of 8, so the block, the swizzle phase key % 8 and the store order are fixed per
+// thread and every address is a per-thread base plus a constant.  All
 // shared-memory loads are issued first.  A 16-byte warp store is served in phases of 8 lanes (one
 // key, all eight blocks): lanes of the second 64-element half store their odd chunk first, so the
 // 8 lanes of a phase hit 8 distinct banks.  Keys >= n (past the run's end) are written as zeros.
-template <bool kFull>
+template <int NT, bool kFull>
 __device__ __forceinline__ void dequant_tile(const uint8_t* pk, uint8_t* dst, int n, int dt) {
-  constexpr int NT = 192, KS = NT / 8;  // 24 keys per pass
-  constexpr int kIt = (BN + KS - 1) / KS;  // 6 passes; the last one only for dt < 64
+  static_assert(NT % 64 == 0, "keys per pass must be a multiple of 8");
+  constexpr int KS = NT / 8;               // keys per pass: 24 for 192 threads, 40 for 320
+  constexpr int kIt = (BN + KS - 1) / KS;  // passes; the last one may cover only part of the keys
   const int blk = dt & 7, kq = dt >> 3;
   const bool swap = blk >= 4;
   const int c0 = (blk & 3) * 2;
@@ -263,9 +265,43 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int m0 = blockIdx.x * (BM * QT);
+  // This CTA's work item: (b, h), first query row m0 and nq query tiles.
+  int bhi, m0, nq;
+  {
+    const int c = blockIdx.x;
+    if (c < p.n_pair_ctas) {
+      const int big = p.pr * (p.pp + 1);
+      int idx;
+      if (c < big || p.pp == 0) {
+        bhi = c / (p.pp + 1);
+        idx = c % (p.pp + 1);
+      } else {
+        bhi = p.pr + (c - big) / p.pp;
+        idx = (c - big) % p.pp;
+      }
+      m0 = idx * 2 * BM;
+      nq = QT;
+    } else {
+      const int c2 = c - p.n_pair_ctas;
+      const int s_big = p.n_qt - 2 * (p.pp + 1), s_small = p.n_qt - 2 * p.pp;
+      const int big = s_big > 0 ? p.pr * s_big : 0;
+      int idx, pairs;
+      if (c2 < big) {
+        bhi = c2 / s_big;
+        idx = c2 % s_big;
+        pairs = p.pp + 1;
+      } else {
+        bhi = p.pr + (c2 - big) / s_small;
+        idx = (c2 - big) % s_small;
+        pairs = p.pp;
+      }
+      m0 = (2 * pairs + idx) * BM;
+      nq = 1;
+    }
+  }
+  const int h = bhi % p.H, b = bhi / p.H;
   const int64_t bh = static_cast<int64_t>(b) * p.H + h;
+  const int n_dq_warps = C::kDequantWarps;
 
   const uint32_t sbase = ptx::smem_u32(smem);
   auto bar = [&](int i) { return sbase + C::oBar + 8 * i; };
@@ -274,14 +310,14 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar(C::bQFull), 1);
-    ptx::mbar_init(bar(C::bQReady), C::kSoftmaxWarps);
+    ptx::mbar_init(bar(C::bQReady), 4 * nq);
     for (int i = 0; i < NPK; ++i) {
       ptx::mbar_init(bar(C::bPkFull + i), 1);
-      ptx::mbar_init(bar(C::bPkEmpty + i), C::kDequantWarps);
+      ptx::mbar_init(bar(C::bPkEmpty + i), n_dq_warps);
     }
     for (int i = 0; i < NST; ++i) {
-      ptx::mbar_init(bar(C::bKFull + i), C::kDequantWarps);
-      ptx::mbar_init(bar(C::bVFull + i), C::kDequantWarps);
+      ptx::mbar_init(bar(C::bKFull + i), n_dq_warps);
+      ptx::mbar_init(bar(C::bVFull + i), n_dq_warps);
       ptx::mbar_init(bar(C::bKEmpty + i), 1);
       ptx::mbar_init(bar(C::bVEmpty + i), 1);
     }
@@ -291,8 +327,6 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       ptx::mbar_init(bar(C::bODone + q), 1);
     }
     ptx::mbar_init(bar(C::bDrain), 1);
-    ptx::mbar_init(bar(C::bTok + 0), 4);
-    ptx::mbar_init(bar(C::bTok + 1), 4);
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::fence_proxy_async_smem();
@@ -311,10 +345,65 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
   // warpgroup's budget change.
   static_assert(QT == 1 || C::kThreads == 512, "register split assumes four warpgroups");
 
+  // Dequantiser role: thread dt of the nthreads threads of the dequant warps.
+  auto dequant_role = [&](int dt) {
+    const int nthreads = 32 * n_dq_warps;
+    const float inv_gv = 1.0f / max_visible_gv(p, bh);
+    // The per-chunk FP32 scales of this (b, h), staged once, so the per-tile column tables are
+    // built from shared memory.
+    const float2* gtab = reinterpret_cast<const float2*>(smem + C::oTab);
+    const bool use_tab = p.C <= kMaxTabChunks;
+    if (use_tab)
+      for (int c = dt; c < p.C; c += nthreads)
+        reinterpret_cast<float2*>(smem + C::oTab)[c] =
+            make_float2(p.k_g[bh * p.C + c] * p.scale_log2, p.v_g[bh * p.C + c] * inv_gv);
+    ptx::named_bar(3, nthreads);
+    bool ok = true;
+    for (int j = 0; j < p.n_tiles && ok; ++j) {
+      const int st = j % NST;
+      int key0, n;
+      tile_keys(p, j, key0, n);
+      for (int t = 0; t < 2 && ok; ++t) {
+        // the stage's previous tile (j - NST) is done with it: K after its QKs, V after its PVs
+        if (j >= NST) ok = waitw(bar((t == 0 ? C::bKEmpty : C::bVEmpty) + st), ((j / NST) - 1) & 1, abort_flag, p.status);
+        if (!ok) break;
+        const int pk = 2 * j + t;
+        const int slot = pk % NPK;
+        ok = waitw(bar(C::bPkFull + slot), (pk / NPK) & 1, abort_flag, p.status);
+        if (!ok) break;
+        const uint8_t* src = smem + C::oPK + slot * PK_BYTES;
+        uint8_t* dst = smem + (t == 0 ? C::oK : C::oV) + st * TILE16;
+        if (n == BN) dequant_tile<C::kDequantThreads, true>(src, dst, n, dt);
+        else dequant_tile<C::kDequantThreads, false>(src, dst, n, dt);
+        if (t == 0 && dt < BN) {  // per-column tables: one thread per key of the tile
+          float* colK = reinterpret_cast<float*>(smem + C::oCol + (j % NCT) * 2 * BN * 4);
+          const bool valid = dt < n;
+          const int c = valid ? (key0 + dt) / p.Lc : 0;
+          const float2 g = !valid ? make_float2(0.0f, 0.0f)
+                           : use_tab ? gtab[c]
+                                     : make_float2(p.k_g[bh * p.C + c] * p.scale_log2, p.v_g[bh * p.C + c] * inv_gv);
+          colK[dt] = g.x;
+          colK[BN + dt] = g.y;
+          if (dt == 0) {
+            const int uniform = (n == BN) && (key0 / p.Lc == (key0 + BN - 1) / p.Lc);
+            *reinterpret_cast<int4*>(smem + C::oInfo + 16 * (j % NCT)) = make_int4(n, uniform, 0, 0);
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive(bar(C::bPkEmpty + slot));
+          ptx::mbar_arrive(bar(t == 0 ? C::bKFull + st : C::bVFull + st));
+        }
+      }
+    }
+  };
+
   if (warp < C::kSoftmaxWarps) {
     // ============================================================ softmax + epilogue
     if constexpr (QT == 2) ptx::setmaxnreg_inc<176>();
     const int qt = warp >> 2;
+    if (qt < nq) {
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + qt * BN;
@@ -370,13 +459,6 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       const int st = j % NST;
       ok = waitw(bar(C::bSFull + qt), j & 1, abort_flag, p.status) &&
            waitw(bar(C::bKFull + st), (j / NST) & 1, abort_flag, p.status);
-      // With two query tiles the two softmax warpgroups take turns (tile 0 of KV tile j, tile 1 of
-      // j, tile 0 of j + 1, ...): each runs with the SM's exponent and conversion units to itself
-      // while the tensor core works on the other tile's products.
-      if (QT == 2 && kTurns && ok) {
-        if (qt == 1) ok = waitw(bar(C::bTok + 0), j & 1, abort_flag, p.status);
-        else if (j > 0) ok = waitw(bar(C::bTok + 1), (j - 1) & 1, abort_flag, p.status);
-      }
       if (!ok) break;
       ptx::tc_fence_after();
       const int ct = j % NCT;
@@ -500,10 +582,6 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
         }
         l_run += la + lb;
       }
-      if (QT == 2 && kTurns) {
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(C::bTok + qt));
-      }
       ptx::tc_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
@@ -547,14 +625,15 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
         }
       }
     }
+    }
   } else {
   if constexpr (QT == 2) ptx::setmaxnreg_dec<80>();
   if (warp == C::kProducerWarp) {
     // ============================================================ TMA producer
     if (lane == 0) {
       ptx::prefetch_tmap(&tmap_q);
-      ptx::mbar_arrive_expect_tx(bar(C::bQFull), QT * TILE16);
-      for (int q = 0; q < QT; ++q)
+      ptx::mbar_arrive_expect_tx(bar(C::bQFull), nq * TILE16);
+      for (int q = 0; q < nq; ++q)
         for (int half = 0; half < 2; ++half)
           ptx::tma_load_4d(sbase + C::oQ + q * TILE16 + half * HALF16, &tmap_q, half * 64, h,
                            m0 + q * BM, b, bar(C::bQFull));
@@ -616,7 +695,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
               waitw(bar(C::bKFull + 0), 0, abort_flag, p.status);
     if (ok) {
       ptx::tc_fence_after();
-      for (int q = 0; q < QT; ++q) issue_qk(q, 0);
+      for (int q = 0; q < nq; ++q) issue_qk(q, 0);
       ptx::mma_commit_w(bar(C::bKEmpty + 0));
     }
     // Per KV tile j: PV(q, j) as soon as softmax q has written P(q, j), then QK(q, j + 1) into the
@@ -624,7 +703,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
     // tile's work while one softmax runs.
     for (int j = 0; j < p.n_tiles && ok; ++j) {
       const int st = j % NST;
-      for (int q = 0; q < QT && ok; ++q) {
+      for (int q = 0; q < nq && ok; ++q) {
         ok = waitw(bar(C::bPFull + q), j & 1, abort_flag, p.status);
         if (ok && q == 0) ok = waitw(bar(C::bVFull + st), (j / NST) & 1, abort_flag, p.status);
         if (!ok) break;
@@ -633,7 +712,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
         const uint32_t tO = tmem + QT * BN + q * D, tP = tmem + q * BN;
         ptx::mma_pv8_w(tO, tP, dV, kIdescPV, j > 0 ? 1u : 0u);
         ptx::mma_commit_w(bar(C::bODone + q));
-        if (q == QT - 1) ptx::mma_commit_w(bar(C::bVEmpty + st));
+        if (q == nq - 1) ptx::mma_commit_w(bar(C::bVEmpty + st));
         if (j + 1 < p.n_tiles) {
           const int st1 = (j + 1) % NST;
           if (q == 0) {
@@ -642,7 +721,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
             ptx::tc_fence_after();
           }
           issue_qk(q, st1);
-          if (q == QT - 1) ptx::mma_commit_w(bar(C::bKEmpty + st1));
+          if (q == nq - 1) ptx::mma_commit_w(bar(C::bKEmpty + st1));
         }
       }
     }
@@ -652,56 +731,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
     __syncwarp();
   } else {
     // ============================================================ dequant warps
-    const int dt = threadIdx.x - C::kDequantWarp0 * 32;
-    const float inv_gv = 1.0f / max_visible_gv(p, bh);
-    // The per-chunk FP32 scales of this (b, h), staged once, so the per-tile column tables are
-    // built from shared memory.
-    const float2* gtab = reinterpret_cast<const float2*>(smem + C::oTab);
-    const bool use_tab = p.C <= kMaxTabChunks;
-    if (use_tab)
-      for (int c = dt; c < p.C; c += C::kDequantThreads)
-        reinterpret_cast<float2*>(smem + C::oTab)[c] =
-            make_float2(p.k_g[bh * p.C + c] * p.scale_log2, p.v_g[bh * p.C + c] * inv_gv);
-    ptx::named_bar(3, C::kDequantThreads);
-    bool ok = true;
-    for (int j = 0; j < p.n_tiles && ok; ++j) {
-      const int st = j % NST;
-      int key0, n;
-      tile_keys(p, j, key0, n);
-      for (int t = 0; t < 2 && ok; ++t) {
-        // the stage's previous tile (j - NST) is done with it: K after its QKs, V after its PVs
-        if (j >= NST) ok = waitw(bar((t == 0 ? C::bKEmpty : C::bVEmpty) + st), ((j / NST) - 1) & 1, abort_flag, p.status);
-        if (!ok) break;
-        const int pk = 2 * j + t;
-        const int slot = pk % NPK;
-        ok = waitw(bar(C::bPkFull + slot), (pk / NPK) & 1, abort_flag, p.status);
-        if (!ok) break;
-        const uint8_t* src = smem + C::oPK + slot * PK_BYTES;
-        uint8_t* dst = smem + (t == 0 ? C::oK : C::oV) + st * TILE16;
-        if (n == BN) dequant_tile<true>(src, dst, n, dt);
-        else dequant_tile<false>(src, dst, n, dt);
-        if (t == 0 && dt < BN) {  // per-column tables: one thread per key of the tile
-          float* colK = reinterpret_cast<float*>(smem + C::oCol + (j % NCT) * 2 * BN * 4);
-          const bool valid = dt < n;
-          const int c = valid ? (key0 + dt) / p.Lc : 0;
-          const float2 g = !valid ? make_float2(0.0f, 0.0f)
-                           : use_tab ? gtab[c]
-                                     : make_float2(p.k_g[bh * p.C + c] * p.scale_log2, p.v_g[bh * p.C + c] * inv_gv);
-          colK[dt] = g.x;
-          colK[BN + dt] = g.y;
-          if (dt == 0) {
-            const int uniform = (n == BN) && (key0 / p.Lc == (key0 + BN - 1) / p.Lc);
-            *reinterpret_cast<int4*>(smem + C::oInfo + 16 * (j % NCT)) = make_int4(n, uniform, 0, 0);
-          }
-        }
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          ptx::mbar_arrive(bar(C::bPkEmpty + slot));
-          ptx::mbar_arrive(bar(t == 0 ? C::bKFull + st : C::bVFull + st));
-        }
-      }
-    }
+    dequant_role(threadIdx.x - C::kDequantWarp0 * 32);
   }
   }
 
@@ -715,7 +745,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
 
 // ------------------------------------------------------------------ host side
 template <int QT>
-cudaError_t launch(const CUtensorMap& tm, const AttnParams& prm, cudaStream_t stream) {
+cudaError_t launch(const CUtensorMap& tm, const AttnParams& prm, int n_single_ctas, cudaStream_t stream) {
   using C = Cfg<QT>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -724,9 +754,51 @@ cudaError_t launch(const CUtensorMap& tm, const AttnParams& prm, cudaStream_t st
                                     C::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  const dim3 grid((prm.Lq + BM * QT - 1) / (BM * QT), prm.H, prm.B);
-  attention_kernel<QT><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tm, prm);
+  attention_kernel<QT><<<prm.n_pair_ctas + n_single_ctas, C::kThreads, C::kSmemBytes, stream>>>(tm, prm);
   return cudaGetLastError();
+}
+
+// Makespan, in units of one two-tile CTA, of p two-tile and s one-tile CTAs dealt in launch order
+// to g SMs (one CTA per SM at a time), a one-tile CTA costing `single` of a two-tile one.
+double makespan(int p, int s, int g, double single) {
+  std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
+  for (int i = 0; i < g; ++i) free_at.push(0.0);
+  double end = 0.0;
+  for (int i = 0; i < p + s; ++i) {
+    const double t = free_at.top() + (i < p ? 1.0 : single);
+    free_at.pop();
+    free_at.push(t);
+    end = std::max(end, t);
+  }
+  return end;
+}
+
+// Splits the n_qt query tiles of each of the bh (batch, head) pairs into tile pairs (two-tile CTAs,
+// the two softmax warpgroups in ping-pong) and single tiles (one-tile CTAs) so that the launch
+// finishes soonest on g SMs: e.g. 444 tiles on 148 SMs as 148 pairs + 148 singles (1.94 units)
+// instead of 222 pairs in two waves (2 units).  Candidates: all pairs, no pairs, whole waves of
+// pairs.
+void plan_work(int n_qt, int bh, int g, AttnParams& prm, int& n_single_ctas) {
+  // Cost of a one-tile CTA relative to a two-tile one, measured on the 1.3B-class layer: the
+  // per-KV-tile dequantisation and MMA chain, which do not shrink with one query tile, dominate.
+  constexpr double kSingle = 0.94;
+  const int max_p = bh * (n_qt / 2), total = bh * n_qt;
+  std::vector<int> cand = {0, max_p};
+  for (int k = 1; k * g <= max_p; ++k) cand.push_back(k * g);
+  int best_p = max_p;
+  double best = makespan(max_p, total - 2 * max_p, g, kSingle);
+  for (int pc : cand) {
+    const double m = makespan(pc, total - 2 * pc, g, kSingle);
+    if (m < best - 1e-9 || (m < best + 1e-9 && pc > best_p)) {
+      best = m;
+      best_p = pc;
+    }
+  }
+  prm.n_qt = n_qt;
+  prm.pp = best_p / bh;
+  prm.pr = best_p % bh;
+  prm.n_pair_ctas = best_p;
+  n_single_ctas = total - 2 * best_p;
 }
 
 }  // namespace
@@ -801,7 +873,13 @@ int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, in
                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return NVFP4KV_ERR_CUDA;
-  const cudaError_t e = q_tokens <= BM ? launch<1>(tm, prm, stream) : launch<2>(tm, prm, stream);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return NVFP4KV_ERR_CUDA;
+  int n_single_ctas = 0;
+  plan_work((q_tokens + BM - 1) / BM, c.batch * c.heads, sms, prm, n_single_ctas);
+  const cudaError_t e = launch<2>(tm, prm, n_single_ctas, stream);
   return e == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 

@@ -30,6 +30,8 @@ constexpr size_t kStaticScratchBytes = 64 * 1024;
 cudaError_t static_scratch_address(void** out);
 cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
                             int64_t token_stride, void* workspace, cudaStream_t stream);
+// Kernels launch_quantize launches for this cache shape on the current device (1 or 2).
+int quantize_launches(const nvfp4kv_cache& c);
 
 // ---- tensor maps (attention.cu): the driver's encoder, looked up once; null if unavailable.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();

@@ -357,6 +357,10 @@ size_t quantize_workspace_bytes(int batch, int heads, int chunk_tokens) {
 
 namespace {
 
+#ifndef NVFP4KV_QUANT_CLUSTER
+#define NVFP4KV_QUANT_CLUSTER 1
+#endif
+
 // Cluster size for the single-pass path, or 0 when the chunk does not fit it: about two CTAs
 // per SM over the whole grid, at least 16 tokens and at most kMaxCtaTokens rows per CTA.
 int cluster_size(int units, int L) {
@@ -366,11 +370,77 @@ int cluster_size(int units, int L) {
   return (L + cl - 1) / cl > kMaxCtaTokens ? 0 : cl;
 }
 
+struct ClusterPlan {
+  int cl = 0;  // 0: the two-pass path
+  int cta_tokens = 0;
+  size_t smem = 0;
+};
+
+cudaLaunchConfig_t cluster_config(const nvfp4kv_cache& c, const ClusterPlan& pl, cudaStream_t stream,
+                                  cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.cl, c.batch * c.heads, 2);
+  cfg.blockDim = dim3(kCThreads, 1, 1);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = pl.cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+// The single-pass plan for this cache shape on the current device, or cl = 0.  The path is only
+// worth taking when every (b, h, tensor) gets its cluster in the first wave (a second wave
+// would wait for the first to finish its whole load-reduce-encode sequence), so the number of
+// co-resident clusters of the shape is asked once per (device, shape).
+ClusterPlan cluster_plan(const nvfp4kv_cache& c) {
+  ClusterPlan pl;
+  const int cl = NVFP4KV_QUANT_CLUSTER ? cluster_size(2 * c.batch * c.heads, c.chunk_tokens) : 0;
+  if (cl == 0 || tensor_map_encoder() == nullptr) return pl;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(quantize_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kMaxCtaTokens * kHeadDim * 2);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(quantize_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  });
+  if (attr_err != cudaSuccess) return pl;
+  ClusterPlan cand;
+  cand.cl = cl;
+  cand.cta_tokens = ((c.chunk_tokens + cl - 1) / cl + kBoxTokens - 1) / kBoxTokens * kBoxTokens;
+  cand.smem = static_cast<size_t>(cand.cta_tokens) * kHeadDim * 2;
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, size_t>, int> active;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return pl;
+  int max_active = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_tuple(dev, cand.cl, cand.smem);
+    auto it = active.find(key);
+    if (it == active.end()) {
+      cudaLaunchAttribute attr[1];
+      const cudaLaunchConfig_t cfg = cluster_config(c, cand, nullptr, attr);
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, quantize_cluster_kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        clusters = 0;
+      }
+      it = active.emplace(key, clusters).first;
+    }
+    max_active = it->second;
+  }
+  return max_active >= 2 * c.batch * c.heads ? cand : pl;
+}
+
 cudaError_t launch_cluster(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
-                           int64_t token_stride, int cl, cudaStream_t stream, bool* launched) {
+                           int64_t token_stride, const ClusterPlan& pl, cudaStream_t stream, bool* launched) {
   *launched = false;
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
-  if (!encode) return cudaSuccess;
   ClusterArgs a;
   a.codes[0] = c.k_codes;
   a.codes[1] = c.v_codes;
@@ -384,7 +454,7 @@ cudaError_t launch_cluster(const nvfp4kv_cache& c, int slot, const uint16_t* k, 
   a.L = c.chunk_tokens;
   a.C = c.capacity_chunks;
   a.slot = slot;
-  a.cta_tokens = ((c.chunk_tokens + cl - 1) / cl + kBoxTokens - 1) / kBoxTokens * kBoxTokens;
+  a.cta_tokens = pl.cta_tokens;
   CUtensorMap tm[2];
   const uint16_t* src[2] = {k, v};
   for (int i = 0; i < 2; ++i) {
@@ -400,51 +470,8 @@ cudaError_t launch_cluster(const nvfp4kv_cache& c, int slot, const uint16_t* k, 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaSuccess;  // not expressible as a tensor map: the two-pass path takes it
   }
-  const size_t smem = static_cast<size_t>(a.cta_tokens) * kHeadDim * 2;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(quantize_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    kMaxCtaTokens * kHeadDim * 2);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(quantize_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  });
-  if (attr_err != cudaSuccess) return cudaSuccess;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cl, c.batch * c.heads, 2);
-  cfg.blockDim = dim3(kCThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cl;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  // How many clusters of this shape can be resident at once, asked once per (device, shape).  The
-  // path is only worth taking when every (b, h, tensor) gets its cluster in the first wave: a
-  // second wave would wait for the first to finish its whole load-reduce-encode sequence.
-  static std::mutex mu;
-  static std::map<std::tuple<int, int, size_t>, int> active;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cudaSuccess;
-  int max_active = 0;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    const auto key = std::make_tuple(dev, cl, smem);
-    auto it = active.find(key);
-    if (it == active.end()) {
-      int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, quantize_cluster_kernel, &cfg) != cudaSuccess) {
-        cudaGetLastError();
-        clusters = 0;
-      }
-      it = active.emplace(key, clusters).first;
-    }
-    max_active = it->second;
-  }
-  if (max_active < 2 * c.batch * c.heads) return cudaSuccess;  // the two-pass path takes it
+  const cudaLaunchConfig_t cfg = cluster_config(c, pl, stream, attr);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_cluster_kernel, tm[0], tm[1], a);
   *launched = e == cudaSuccess;
   return e;
@@ -452,15 +479,14 @@ cudaError_t launch_cluster(const nvfp4kv_cache& c, int slot, const uint16_t* k, 
 
 }  // namespace
 
+int quantize_launches(const nvfp4kv_cache& c) { return cluster_plan(c).cl > 0 ? 1 : 2; }
+
 cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
                             int64_t token_stride, void* workspace, cudaStream_t stream) {
-#ifndef NVFP4KV_QUANT_CLUSTER
-#define NVFP4KV_QUANT_CLUSTER 1
-#endif
-  const int cl = NVFP4KV_QUANT_CLUSTER ? cluster_size(2 * c.batch * c.heads, c.chunk_tokens) : 0;
-  if (cl > 0) {
+  const ClusterPlan pl = cluster_plan(c);
+  if (pl.cl > 0) {
     bool launched = false;
-    const cudaError_t e = launch_cluster(c, slot, k, v, token_stride, cl, stream, &launched);
+    const cudaError_t e = launch_cluster(c, slot, k, v, token_stride, pl, stream, &launched);
     if (launched || e != cudaSuccess) return e;
   }
   QuantArgs a;

@@ -104,6 +104,8 @@ def test_dequantize_and_status_argument_checks(L):
     assert L.nvfp4_kv_dequantize(ctypes.byref(d), 0, 3, 2, 0x90000, None) == nk.ERR_INVALID_ARG
     assert L.nvfp4_kv_dequantize(ctypes.byref(d), 0, 0, 1, 0x90008, None) == nk.ERR_INVALID_ARG
     assert L.nvfp4kv_read_status(None, None, None) == nk.ERR_INVALID_ARG
+    assert L.nvfp4kv_quantize_launches(None) == -nk.ERR_INVALID_ARG
+    assert L.nvfp4kv_quantize_launches(ctypes.byref(_desc(head_dim=256))) == -nk.ERR_UNSUPPORTED
     assert L.nvfp4kv_debug_encode(None, 4, 0x1000, 0x2000, None) == nk.ERR_INVALID_ARG
     assert L.nvfp4kv_workspace_bytes(None, 64) == 0
     assert L.nvfp4kv_workspace_bytes(ctypes.byref(d), 64) >= 256
@@ -115,6 +117,7 @@ def test_valid_arguments_without_a_gpu_report_a_cuda_error(L):
         pytest.skip("a GPU is present")
     assert _quant(L, _desc()) == nk.ERR_CUDA
     assert _attn(L, _desc()) == nk.ERR_CUDA
+    assert L.nvfp4kv_quantize_launches(ctypes.byref(_desc())) == -nk.ERR_CUDA
 
 
 def test_strerror_covers_every_code(L):

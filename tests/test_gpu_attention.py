@@ -52,6 +52,10 @@ EDGE = {
     # query chunk at slot 0
     "first_chunk": dict(batch=1, heads=2, chunk_tokens=256, capacity=3, q_chunk=0, n_sink=1, window=3,
                         q_tokens=256),
+    # 148 heads of two query tiles (128 + 72 rows): one two-tile CTA per head on a 148-SM B200,
+    # so the ragged tile sits in the second softmax warpgroup
+    "ragged_pairs": dict(batch=1, heads=148, chunk_tokens=64, capacity=3, q_chunk=2, n_sink=1, window=2,
+                         q_tokens=200),
 }
 
 

@@ -71,13 +71,14 @@ def test_special_chunks_match_oracle(name, path):
              "ties0": lambda: sc.tie_chunk(0), "ties-9": lambda: sc.tie_chunk(-9),
              "underflow": sc.underflow_chunk, "tiny_scale": sc.tiny_scale_chunk}[name]()
     chunk = sc.pad_tokens(chunk)
-    if path == "two_pass":
+    if path == "two_pass":  # long enough that no cluster holds a (b, h, tensor) in shared memory
         reps = -(-TWO_PASS_TOKENS // chunk.shape[1])
         chunk = np.ascontiguousarray(np.tile(chunk, (1, reps, 1, 1)))
     L = chunk.shape[1]
     cache = KVCache(1, 1, L, 2)
     ocache = oracle.Cache(1, 1, 128, L, 2)
     neg = chunk ^ np.uint16(0x8000)  # V gets the negated chunk
+    assert cache.quantize_launches() == (1 if path == "cluster" else 2)
     cache.quantize(1, dev_bf16(chunk), dev_bf16(neg))
     ocache.append(1, chunk, neg)
     assert_cache_equal(cache, ocache, [1])
@@ -88,6 +89,7 @@ def test_special_chunks_match_oracle(name, path):
 def test_long_chunk_two_pass_path_matches_oracle():
     w = dataclasses.replace(synthetic.WORKLOADS["tiny"], heads=2, chunk_tokens=TWO_PASS_TOKENS + 8, capacity=2)
     cache, ocache = make_caches(w, [1])
+    assert cache.quantize_launches() == 2
     assert_cache_equal(cache, ocache, [1])
     assert cache.read_status() == 0
 
