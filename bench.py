@@ -320,15 +320,16 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "dtype_detail": "cache NVFP4 (E2M1 + E4M3 + fp32); QK^T bf16 x bf16 and PV fp16 x fp16 "
-                            "on tcgen05 with fp32 accumulate; fp32 output",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
+            "dtype_detail": "bf16 Q/K/V in; cache NVFP4 (E2M1 + E4M3 + fp32); QK^T and PV fp16 x fp16 "
+                            "(exact conversions of the bf16 query and the dequantised K/V) on tcgen05 "
+                            "with fp32 accumulate; fp32 output",
             "data": "synthetic (seeded N(0,1) with outlier channels; no dataset or weights)",
             "config": config_of(w),
             "roofline": {"bound": "tensor", "kernel": "attention_kernel", "achieved": attn_tflops,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": attn_tflops / peaks["bf16_tflops"], "traffic": traffic,
-                         "peak_source": f"{src} bf16 burst (cuBLAS 8192^3)",
+                         "peak_source": f"{src} bf16 burst (cuBLAS 8192^3); fp16 has the same nominal tensor rate",
                          "algorithmic_flops_per_launch": attn_flops,
                          "algorithmic_bytes_per_launch": attn_bytes,
                          "launch_us": t_attn * 1e3},

@@ -7,22 +7,25 @@
 // 2.1: a chunk sees its own tokens.  Reading note (yingwang.github.io), "The NVFP4
 // quantization format": x_hat = E2M1 * E4M3 * FP32 scale.
 //
-// One CTA owns QT query tiles of 128 rows of one (batch, head) and walks the visible KV
-// tiles (128 keys each; tiles lie inside runs of consecutive visible chunks, so chunks
-// outside the mask are never read).  Warp roles:
-//   softmax warps [0, 4*QT)   one query row per thread, online softmax over TMEM rows
-//   producer warp             TMA: Q tiles (tensor map, 128B swizzle) and packed K/V tiles
+// One CTA owns one or two query tiles of 128 rows of one (batch, head) and walks the visible
+// KV tiles (128 keys each; tiles lie inside runs of consecutive visible chunks, so chunks
+// outside the mask are never read).  A host planner chooses how many CTAs take two tiles.
+// 512 threads, four warpgroups; warp roles:
+//   softmax warps 0-3, 4-7    query tile 0 / 1: one query row per thread, online softmax over
+//                             TMEM rows, epilogue (176 registers each, setmaxnreg)
+//   producer warp 8           TMA: Q tiles (tensor map, 128B swizzle) and packed K/V tiles
 //                             + E4M3 scales (1-D bulk copies) into a ring of smem slots
-//   MMA warp                  TMEM allocation; tcgen05.mma S = Q K^T (both operands in
-//                             smem), O += P V (P from TMEM, V from smem)
-//   dequant warps (4)         E2M1 * E4M3 products, exact in 16 bits, written straight
-//                             into the 128B-swizzled UMMA operand layout: bf16 K (the
-//                             B operand of Q K^T, K-major) and fp16 V (the B operand of
-//                             P V, MN-major)
-// The FP32 scales stay out of the MMAs: g_K(chunk) multiplies S per column, and
-// g_V(chunk) / max g_V multiplies P per column before P is rounded to fp16 (fp16 P and V
-// keep the P V product 8x finer than bf16).  Rows are rescaled lazily: the running max
-// only moves when it grows by more than 2^8.
+//   MMA warp 9                TMEM allocation; tcgen05.mma S = Q K^T (both operands in
+//                             smem), O += P V (P from TMEM, V from smem), eight MMAs per asm
+//                             block from one elected lane
+//   dequant warps 10-15       E2M1 * E4M3 products, exact in fp16, written straight into the
+//                             128B-swizzled UMMA operand layout: K (the B operand of Q K^T,
+//                             K-major) and V (the B operand of P V, MN-major)
+// With two tiles the softmax warpgroups alternate with the tensor core: PV(0, j), QK(0, j+1),
+// PV(1, j), QK(1, j+1).  The FP32 scales stay out of the MMAs: g_K(chunk) multiplies S per
+// column, and g_V(chunk) / max g_V multiplies P per column before P is rounded to fp16 (fp16
+// P and V keep the P V product 8x finer than bf16).  Rows are rescaled lazily: the running
+// max only moves when it grows by more than 2^8.
 //
 // Every mbarrier wait is bounded (%globaltimer); on a time-out the kernel ORs
 // NVFP4KV_ERR_DEVICE_TIMEOUT into the status word, lets in-flight copies and MMAs finish,
@@ -55,10 +58,6 @@ constexpr int PK_BYTES = PK_CODES + BN * kScaleBytes;   // 9216
 constexpr int TILE16 = BN * D * 2;                      // one 128 x 128 16-bit operand tile
 constexpr int HALF16 = TILE16 / 2;                      // 128 rows x 64 elements (128 B rows)
 constexpr int MAX_RUNS = 4;
-#ifndef NVFP4KV_EXP2_EMUL
-#define NVFP4KV_EXP2_EMUL 0
-#endif
-constexpr int kExp2Emul = NVFP4KV_EXP2_EMUL;  // 0: every exponent on the MUFU
 
 template <int QT>
 struct Cfg {
@@ -537,8 +536,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       // all-zero V chunk (cv = 0) adds 0 to O and its p to l.
       float la = 0.0f, lb = 0.0f;
       if (uni) {
-        // x = S * ck + log2(cv) - m in packed pairs; one exponent in 2 * kExp2Emul is taken on the
-        // FMA pipe (ex2_poly3) to relieve the MUFU; eight independent row-sum chains.
+        // x = S * ck + log2(cv) - m in packed pairs; eight independent row-sum chains.
         const float mneg = log2f(colV[0]) - m_run;
         float l8[8];
 #pragma unroll
@@ -550,8 +548,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
           for (int i = 0; i < 16; ++i) {
             float x0, x1;
             ptx::ffma2(x0, x1, __uint_as_float(sr[c][2 * i]), __uint_as_float(sr[c][2 * i + 1]), ck, mneg);
-            const bool emul = kExp2Emul > 0 && (i % (kExp2Emul > 0 ? kExp2Emul : 1)) == kExp2Emul - 1;
-            pk[i] = ptx::f32x2_to_f16x2(emul ? ptx::ex2_poly3(x0) : ptx::ex2(x0), ptx::ex2(x1));
+            pk[i] = ptx::f32x2_to_f16x2(ptx::ex2(x0), ptx::ex2(x1));
             l8[i & 7] = ptx::add_f16x2_f32(l8[i & 7], pk[i]);
           }
           ptx::tmem_st16p(tS + 16 * c, pk);

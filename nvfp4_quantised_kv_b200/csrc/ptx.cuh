@@ -474,20 +474,6 @@ __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
 
-// 2^x on the FMA pipe, for x <= 2^20: x = n + f with n = round(x) (the 1.5 * 2^23 shift leaves n
-// in the low mantissa bits) and f in [-1/2, 1/2]; 2^f by a cubic fitted to minimum maximum relative
-// error on that interval (Lawson's iteration; max relative error 7.5e-5, below half an fp16 ulp);
-// n is added to the exponent field.  Inputs below -125 return 2^-125 * 2^f (far below fp16 range).
-constexpr float kExp2C0 = 0.99992811f, kExp2C1 = 0.69326099f, kExp2C2 = 0.24261054f,
-                kExp2C3 = 0.05517132f;
-__device__ __forceinline__ float ex2_poly3(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -223,10 +223,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const __grid_constan
 constexpr int kBoxTokens = 16;          // tokens per TMA box (16 x 256 B)
 constexpr int kMaxCtaTokens = 448;      // 112 KB of bf16 rows: two CTAs per SM
 constexpr int kMaxCluster = 16;
-#ifndef NVFP4KV_QC_THREADS
-#define NVFP4KV_QC_THREADS 512
-#endif
-constexpr int kCThreads = NVFP4KV_QC_THREADS;
+constexpr int kCThreads = 512;
 constexpr int kCWarps = kCThreads / 32;
 
 struct ClusterArgs {
@@ -357,10 +354,6 @@ size_t quantize_workspace_bytes(int batch, int heads, int chunk_tokens) {
 
 namespace {
 
-#ifndef NVFP4KV_QUANT_CLUSTER
-#define NVFP4KV_QUANT_CLUSTER 1
-#endif
-
 // Cluster size for the single-pass path, or 0 when the chunk does not fit it: about two CTAs
 // per SM over the whole grid, at least 16 tokens and at most kMaxCtaTokens rows per CTA.
 int cluster_size(int units, int L) {
@@ -398,7 +391,7 @@ cudaLaunchConfig_t cluster_config(const nvfp4kv_cache& c, const ClusterPlan& pl,
 // co-resident clusters of the shape is asked once per (device, shape).
 ClusterPlan cluster_plan(const nvfp4kv_cache& c) {
   ClusterPlan pl;
-  const int cl = NVFP4KV_QUANT_CLUSTER ? cluster_size(2 * c.batch * c.heads, c.chunk_tokens) : 0;
+  const int cl = cluster_size(2 * c.batch * c.heads, c.chunk_tokens);
   if (cl == 0 || tensor_map_encoder() == nullptr) return pl;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
