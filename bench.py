@@ -160,6 +160,28 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings over all ranks (identity on one process): a
+    multi-GPU number is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor(list(values), device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(units_per_rank, world, ms_per_step):
+    """Whole-job throughput: the units all ranks processed per second of the slowest rank."""
+    return units_per_rank * world / (ms_per_step * 1e-3)
+
+
+def replica_seed(seed, rotation, rank):
+    """Seed of one rotating input set of one rank: every replica draws its own inputs."""
+    return seed + 1000 * rotation + 7919 * rank
+
+
 def config_of(w):
     return {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
             "chunk_tokens": w.chunk_tokens, "q_tokens": w.q_tokens, "visible_keys": w.visible_tokens,
@@ -210,7 +232,7 @@ def main():
     sets = []
     hist = [c for c in w.visible_chunks if c != w.q_chunk]
     for s in range(ROTATE):
-        ws = synthetic.Workload(**{**w.__dict__, "seed": w.seed + 1000 * s + 7919 * rank})
+        ws = synthetic.Workload(**{**w.__dict__, "seed": replica_seed(w.seed, s, rank)})
         cache = nk.KVCache(w.batch, w.heads, w.chunk_tokens, w.capacity, q_tokens_max=w.q_tokens, device=dev)
         for slot in hist:
             k, v = synthetic.chunk_kv(ws, slot)
@@ -258,10 +280,7 @@ def main():
     elapsed_ms = start.elapsed_time(end)
     t_quant = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     t_attn = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) / w.attn_calls
-    if world > 1:
-        t = torch.tensor([elapsed_ms, t_quant, t_attn], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, t_quant, t_attn = t.tolist()
+    elapsed_ms, t_quant, t_attn = max_over_ranks([elapsed_ms, t_quant, t_attn], dev)
     for S in sets:
         assert S["cache"].read_status() == 0, "device status set during the timed region"
 
@@ -294,17 +313,15 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    (e2e_ms,) = max_over_ranks([e2e_ms], dev)
     if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
         dist.barrier()
 
     attn_flops, attn_bytes, quant_bytes = work(w)
     q_launches = sets[0]["cache"].quantize_launches()
     ms_per_step = elapsed_ms / args.steps
     step_flops = attn_flops * w.attn_calls
-    value = step_flops * world / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_rate(step_flops, world, ms_per_step) / 1e12
     peaks, src = load_peaks()
     attn_tflops = attn_flops / (t_attn * 1e-3) / 1e12
     quant_gbs = quant_bytes / (t_quant * 1e-3) / 1e9
@@ -339,7 +356,7 @@ def main():
                          "achieved": quant_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": quant_gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_call": quant_bytes,
                          "call_us": t_quant * 1e3, "peak_source": f"{src} HBM copy"},
-            "e2e": {"value": step_flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": whole_job_rate(step_flops, world, e2e_ms) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": args.steps * (q_launches + w.attn_calls),
             "clocks": clk,
