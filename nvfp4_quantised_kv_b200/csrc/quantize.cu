@@ -39,6 +39,10 @@ constexpr int kWarps = kThreads / 32;
 // before it uses any (one memory latency per CTA).
 constexpr int kPasses = 8;
 constexpr int kPartTokens = (kThreads / 16) * kPasses;  // 128
+// The encode pass holds fewer rows per CTA (it also keeps the encoder state): 64 tokens, so both
+// grids run six CTAs per SM and more, smaller CTAs shorten the tail.
+constexpr int kEncPasses = 4;
+constexpr int kEncTokens = (kThreads / 16) * kEncPasses;  // 64
 
 struct QuantArgs {
   const uint16_t* x[2];  // K, V (bf16 bits)
@@ -133,7 +137,7 @@ __device__ __forceinline__ void encode_store(uint4 w, const Encoder& e, const fl
   }
 }
 
-__global__ void __launch_bounds__(kThreads) amax_kernel(const __grid_constant__ QuantArgs a) {
+__global__ void __launch_bounds__(kThreads, 6) amax_kernel(const __grid_constant__ QuantArgs a) {
   const int part = blockIdx.x, bh = blockIdx.y, tensor = blockIdx.z;
   const int b = bh / a.H, h = bh % a.H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -166,20 +170,20 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const __grid_constant__ 
   }
 }
 
-__global__ void __launch_bounds__(kThreads) quantize_kernel(const __grid_constant__ QuantArgs a) {
+__global__ void __launch_bounds__(kThreads, 6) quantize_kernel(const __grid_constant__ QuantArgs a) {
   const int part = blockIdx.x, bh = blockIdx.y, tensor = blockIdx.z;
   const int b = bh / a.H, h = bh % a.H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t_begin = part * kPartTokens;
-  const int t_end = min(a.L, t_begin + kPartTokens);
+  const int t_begin = part * kEncTokens;
+  const int t_end = min(a.L, t_begin + kEncTokens);
   const int sub = threadIdx.x >> 4;
   const uint16_t* x = a.x[tensor] + static_cast<int64_t>(b) * a.L * a.token_stride +
                       static_cast<int64_t>(h) * kHeadDim + (threadIdx.x & 15) * 8;
   // The rows do not depend on the amax grid: they are loaded (mostly from L2, where that grid
   // just read them) before waiting for its partial maxima.
-  uint4 w[kPasses];
+  uint4 w[kEncPasses];
 #pragma unroll
-  for (int u = 0; u < kPasses; ++u) {
+  for (int u = 0; u < kEncPasses; ++u) {
     const int t = t_begin + u * (kThreads / 16) + sub;
     w[u] = t < t_end ? ld_row16(x + static_cast<int64_t>(t) * a.token_stride) : make_uint4(0, 0, 0, 0);
   }
@@ -208,7 +212,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const __grid_constan
   uint8_t* codes = a.codes[tensor] + row0 * kCodeBytes + (lane & 15) * 4;
   uint8_t* scales = a.scales[tensor] + row0 * kScaleBytes + ((lane & 15) >> 1);
 #pragma unroll
-  for (int u = 0; u < kPasses; ++u) {
+  for (int u = 0; u < kEncPasses; ++u) {
     const int t = t_begin + u * (kThreads / 16) + sub;
     encode_store(w[u], enc, rtab, t < t_end, codes + static_cast<int64_t>(t) * kCodeBytes,
                  scales + static_cast<int64_t>(t) * kScaleBytes, lane);
@@ -507,7 +511,7 @@ cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k,
   // The encode grid is a programmatic dependent of the amax grid: it launches while the amax grid
   // drains and waits (griddepcontrol.wait) only before it reads the partial maxima.
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
+  cfg.gridDim = dim3((c.chunk_tokens + kEncTokens - 1) / kEncTokens, c.batch * c.heads, 2);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
