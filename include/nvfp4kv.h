@@ -161,6 +161,16 @@ int nvfp4_kv_dequantize(const nvfp4kv_cache* cache, int32_t which, int32_t first
 int nvfp4kv_debug_encode(const float* x, int64_t n, uint8_t* e2m1_codes, uint8_t* e4m3_codes,
                          void* cuda_stream);
 
+/* The work split nvfp4_kv_attention uses for q_tokens queries on n_sms SMs (n_sms <= 0: the
+ * current device's count; any n_sms > 0 needs no GPU).  out[0] = number of CTAs; for 0 <= cta <
+ * out[0] also that CTA's work item: out[1] = b * heads + h, out[2] = first query row, out[3] =
+ * query tiles of 128 rows (1 or 2, clipped to q_tokens by the kernel).  A host planner chooses how
+ * many CTAs take two tiles so that the launch finishes soonest.  A library diagnostic with no
+ * counterpart in the pages.  Errors: NVFP4KV_ERR_INVALID_ARG (bad cache, q_tokens <= 0, null out,
+ * cta >= out[0]), NVFP4KV_ERR_CUDA (n_sms <= 0 without a device). */
+int nvfp4kv_attention_plan(const nvfp4kv_cache* cache, int32_t q_tokens, int32_t n_sms, int32_t cta,
+                           int32_t* out);
+
 /* Kernels that nvfp4_kv_quantize (and its static-scratch variant) launch per call for this cache
  * shape on the current device: 1 when every (batch, head, tensor) gets one thread-block cluster
  * in a single wave (single pass: the input crosses HBM once), 2 otherwise (an amax pass and an

@@ -51,6 +51,7 @@ SIGNATURES = {
     "nvfp4_kv_dequantize": (ctypes.c_int, [_CP, _i32, _i32, _i32, _vp, _vp]),
     "nvfp4kv_debug_encode": (ctypes.c_int, [_vp, _i64, _vp, _vp, _vp]),
     "nvfp4kv_quantize_launches": (ctypes.c_int, [_CP]),
+    "nvfp4kv_attention_plan": (ctypes.c_int, [_CP, _i32, _i32, _i32, ctypes.POINTER(_i32)]),
     "nvfp4kv_read_status": (ctypes.c_int, [_CP, _vp, ctypes.POINTER(ctypes.c_uint32)]),
     "nvfp4kv_strerror": (ctypes.c_char_p, [ctypes.c_int]),
 }

@@ -158,6 +158,23 @@ int nvfp4kv_debug_encode(const float* x, int64_t n, uint8_t* e2m1_codes, uint8_t
   return e == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 
+int nvfp4kv_attention_plan(const nvfp4kv_cache* cache, int32_t q_tokens, int32_t n_sms, int32_t cta,
+                           int32_t* out) {
+  int rc = check_cache(cache);
+  if (rc != NVFP4KV_OK) return rc;
+  if (q_tokens <= 0 || !out) return NVFP4KV_ERR_INVALID_ARG;
+  if (n_sms <= 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return NVFP4KV_ERR_CUDA;
+  }
+  int o[4];
+  rc = attention_plan(*cache, q_tokens, n_sms, cta, o);
+  for (int i = 0; i < 4; ++i) out[i] = o[i];
+  return rc;
+}
+
 int nvfp4kv_quantize_launches(const nvfp4kv_cache* cache) {
   int rc = check_cache(cache);
   if (rc != NVFP4KV_OK) return -rc;

@@ -255,6 +255,48 @@ __device__ __forceinline__ void dequant_tile(const uint8_t* pk, uint8_t* dst, in
   }
 }
 
+// Work item of CTA c: every (b, h) has n_qt query tiles; (b, h) < pr gives its first pp + 1 tile
+// pairs to two-tile CTAs, the others their first pp; CTAs [0, n_pair_ctas) take those pairs in
+// (b, h) order, the rest take the remaining tiles one by one, also in (b, h) order.  Shared by the
+// kernel and the host diagnostic that checks the split.
+struct WorkItem {
+  int bhi, m0, nq;
+};
+
+__host__ __device__ inline WorkItem work_item(int c, int n_qt, int pp, int pr, int n_pair_ctas) {
+  WorkItem w;
+  if (c < n_pair_ctas) {
+    const int big = pr * (pp + 1);
+    int idx;
+    if (c < big || pp == 0) {
+      w.bhi = c / (pp + 1);
+      idx = c % (pp + 1);
+    } else {
+      w.bhi = pr + (c - big) / pp;
+      idx = (c - big) % pp;
+    }
+    w.m0 = idx * 2 * BM;
+    w.nq = 2;
+  } else {
+    const int c2 = c - n_pair_ctas;
+    const int s_big = n_qt - 2 * (pp + 1), s_small = n_qt - 2 * pp;
+    const int big = s_big > 0 ? pr * s_big : 0;
+    int idx, pairs;
+    if (c2 < big || s_small <= 0) {
+      w.bhi = s_big > 0 ? c2 / s_big : 0;
+      idx = s_big > 0 ? c2 % s_big : 0;
+      pairs = pp + 1;
+    } else {
+      w.bhi = pr + (c2 - big) / s_small;
+      idx = (c2 - big) % s_small;
+      pairs = pp;
+    }
+    w.m0 = (2 * pairs + idx) * BM;
+    w.nq = 1;
+  }
+  return w;
+}
+
 template <int QT>
 __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ AttnParams p) {
@@ -265,39 +307,8 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   // This CTA's work item: (b, h), first query row m0 and nq query tiles.
-  int bhi, m0, nq;
-  {
-    const int c = blockIdx.x;
-    if (c < p.n_pair_ctas) {
-      const int big = p.pr * (p.pp + 1);
-      int idx;
-      if (c < big || p.pp == 0) {
-        bhi = c / (p.pp + 1);
-        idx = c % (p.pp + 1);
-      } else {
-        bhi = p.pr + (c - big) / p.pp;
-        idx = (c - big) % p.pp;
-      }
-      m0 = idx * 2 * BM;
-      nq = QT;
-    } else {
-      const int c2 = c - p.n_pair_ctas;
-      const int s_big = p.n_qt - 2 * (p.pp + 1), s_small = p.n_qt - 2 * p.pp;
-      const int big = s_big > 0 ? p.pr * s_big : 0;
-      int idx, pairs;
-      if (c2 < big) {
-        bhi = c2 / s_big;
-        idx = c2 % s_big;
-        pairs = p.pp + 1;
-      } else {
-        bhi = p.pr + (c2 - big) / s_small;
-        idx = (c2 - big) % s_small;
-        pairs = p.pp;
-      }
-      m0 = (2 * pairs + idx) * BM;
-      nq = 1;
-    }
-  }
+  const WorkItem wi = work_item(blockIdx.x, p.n_qt, p.pp, p.pr, p.n_pair_ctas);
+  const int bhi = wi.bhi, m0 = wi.m0, nq = wi.nq;
   const int h = bhi % p.H, b = bhi / p.H;
   const int64_t bh = static_cast<int64_t>(b) * p.H + h;
   const int n_dq_warps = C::kDequantWarps;
@@ -815,6 +826,22 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 size_t attention_workspace_bytes(const nvfp4kv_cache&, int) { return 0; }
+
+int attention_plan(const nvfp4kv_cache& c, int q_tokens, int n_sms, int cta, int out[4]) {
+  AttnParams prm{};
+  int n_single = 0;
+  const int n_qt = (q_tokens + BM - 1) / BM;
+  plan_work(n_qt, c.batch * c.heads, n_sms, prm, n_single);
+  out[0] = prm.n_pair_ctas + n_single;
+  out[1] = out[2] = out[3] = 0;
+  if (cta < 0) return NVFP4KV_OK;
+  if (cta >= out[0]) return NVFP4KV_ERR_INVALID_ARG;
+  const WorkItem w = work_item(cta, prm.n_qt, prm.pp, prm.pr, prm.n_pair_ctas);
+  out[1] = w.bhi;
+  out[2] = w.m0;
+  out[3] = w.nq;
+  return NVFP4KV_OK;
+}
 
 int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, int64_t q_stride,
                      int q_chunk, int n_sink, int window, float softmax_scale, void* out,

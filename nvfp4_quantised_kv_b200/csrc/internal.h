@@ -38,6 +38,9 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // ---- attention (attention.cu)
 size_t attention_workspace_bytes(const nvfp4kv_cache& c, int q_tokens);
+// The attention launch's work split for n_sms SMs: out[0] = CTAs; for cta >= 0 also its work item
+// out[1] = batch * heads + head index, out[2] = first query row, out[3] = query tiles (1 or 2).
+int attention_plan(const nvfp4kv_cache& c, int q_tokens, int n_sms, int cta, int out[4]);
 int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, int64_t q_stride,
                      int q_chunk, int n_sink, int window, float softmax_scale, void* out,
                      int out_dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream);
