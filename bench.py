@@ -349,6 +349,7 @@ def main():
                          "peak_source": f"{src} bf16 burst (cuBLAS 8192^3); fp16 has the same nominal tensor rate",
                          "algorithmic_flops_per_launch": attn_flops,
                          "algorithmic_bytes_per_launch": attn_bytes,
+                         "algorithmic_hbm_gbs": attn_bytes / (t_attn * 1e-3) / 1e9,
                          "launch_us": t_attn * 1e3},
             "quantize": {"bound": "hbm",
                          "kernels": ("quantize_cluster_kernel" if q_launches == 1
