@@ -49,6 +49,13 @@ def lib() -> ctypes.CDLL:
             [ctypes.c_void_p] + [ctypes.c_int32] * 4 + [ctypes.c_int64] + [ctypes.c_void_p] * 6 +
             [ctypes.c_int32] * 5 + [ctypes.c_double, ctypes.c_void_p, ctypes.c_int32,
                                     ctypes.c_void_p])
+        L.oracle_multishot_chunks.restype = ctypes.c_int
+        L.oracle_multishot_chunks.argtypes = [ctypes.c_int32] * 6 + [ctypes.c_void_p]
+        L.oracle_attention_rows_slots.restype = ctypes.c_int
+        L.oracle_attention_rows_slots.argtypes = (
+            [ctypes.c_void_p] + [ctypes.c_int32] * 4 + [ctypes.c_int64] + [ctypes.c_void_p] * 6 +
+            [ctypes.c_int32] * 2 + [ctypes.c_void_p, ctypes.c_int32, ctypes.c_double, ctypes.c_void_p,
+                                    ctypes.c_int32, ctypes.c_void_p])
         del u8p
         _LIB = L
     return _LIB
@@ -146,6 +153,34 @@ def visible_chunks(q_chunk: int, n_sink: int, window: int, capacity: int) -> lis
     if n < 0:
         raise ValueError("oracle_visible_chunks rejected its arguments")
     return [int(c) for c in out[:n]]
+
+
+def multishot_chunks(q_chunk: int, n_sink: int, window: int, shot_start: int, shot_len: int,
+                     capacity: int) -> list[int]:
+    """Global sink U shot sink (start, len) U sliding window, each chunk once, ascending."""
+    out = np.zeros(max(capacity, 1), np.int32)
+    n = lib().oracle_multishot_chunks(q_chunk, n_sink, window, shot_start, shot_len, capacity, _ptr(out))
+    if n < 0:
+        raise ValueError("oracle_multishot_chunks rejected its arguments")
+    return [int(c) for c in out[:n]]
+
+
+def attention_rows_slots(q_bf16: np.ndarray, cache: Cache, slots, rows: np.ndarray,
+                         softmax_scale: float = 0.0) -> np.ndarray:
+    """fp64 attention of ``rows`` over the keys of the listed chunk slots (union, any order)."""
+    q = np.ascontiguousarray(q_bf16, dtype=np.uint16)
+    B, Lq, H, d = q.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int32).reshape(-1, 3)
+    sl = np.ascontiguousarray(slots, dtype=np.int32).reshape(-1)
+    out = np.zeros((rows.shape[0], d), np.float64)
+    c = cache
+    rc = lib().oracle_attention_rows_slots(
+        _ptr(q), B, Lq, H, d, H * d, _ptr(c.k_codes), _ptr(c.k_scales), _ptr(c.k_g),
+        _ptr(c.v_codes), _ptr(c.v_scales), _ptr(c.v_g), c.Lc, c.C, _ptr(sl), sl.shape[0],
+        float(softmax_scale), _ptr(rows), rows.shape[0], _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_attention_rows_slots rejected its arguments")
+    return out
 
 
 def attention_rows(q_bf16: np.ndarray, cache: Cache, q_chunk: int, n_sink: int, window: int,

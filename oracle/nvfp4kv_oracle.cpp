@@ -210,20 +210,38 @@ int oracle_visible_chunks(int32_t q_chunk, int32_t n_sink, int32_t window, int32
   return n;
 }
 
-int oracle_attention_rows(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, int32_t d,
-                          int64_t q_token_stride,
-                          const uint8_t* k_codes, const uint8_t* k_scales, const float* k_gscale,
-                          const uint8_t* v_codes, const uint8_t* v_scales, const float* v_gscale,
-                          int32_t chunk_tokens, int32_t capacity,
-                          int32_t q_chunk, int32_t n_sink, int32_t window, double softmax_scale,
-                          const int32_t* rows, int32_t n_rows, double* out) {
+int oracle_multishot_chunks(int32_t q_chunk, int32_t n_sink, int32_t window, int32_t shot_start,
+                            int32_t shot_len, int32_t capacity, int32_t* out) {
+  /* the shot sink is the start of the current shot: history, never past the query chunk */
+  if (!out || capacity <= 0 || q_chunk < 0 || q_chunk >= capacity || n_sink < 0 || window < 1 ||
+      shot_start < 0 || shot_len < 0 || shot_start + shot_len > q_chunk + 1)
+    return -1;
+  int n = 0;
+  for (int32_t c = 0; c < capacity; ++c) {
+    const bool global_sink = c < n_sink;                                  /* A_g */
+    const bool shot_sink = c >= shot_start && c < shot_start + shot_len;  /* A_s = (start, len) */
+    const bool in_window = (c > q_chunk - window) && (c <= q_chunk);      /* sliding window */
+    if (global_sink || shot_sink || in_window) out[n++] = c;             /* union, each chunk once */
+  }
+  return n;
+}
+
+}  // extern "C"
+
+namespace {
+
+/* fp64 attention of the requested rows over the keys of the chunk slots vis[0..nvis) (ascending,
+ * distinct): the plain definition, two passes per row. */
+int attention_over_slots(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, int32_t d,
+                         int64_t q_token_stride,
+                         const uint8_t* k_codes, const uint8_t* k_scales, const float* k_gscale,
+                         const uint8_t* v_codes, const uint8_t* v_scales, const float* v_gscale,
+                         int32_t chunk_tokens, int32_t capacity, const int32_t* vis, int nvis,
+                         double softmax_scale, const int32_t* rows, int32_t n_rows, double* out) {
   if (!q || !k_codes || !k_scales || !k_gscale || !v_codes || !v_scales || !v_gscale || !rows ||
       !out || B <= 0 || Lq <= 0 || H <= 0 || d <= 0 || d % 16 != 0 || chunk_tokens <= 0 ||
-      capacity <= 0 || n_rows < 0 || q_token_stride < static_cast<int64_t>(H) * d)
+      capacity <= 0 || n_rows < 0 || q_token_stride < static_cast<int64_t>(H) * d || nvis < 0)
     return -1;
-  std::vector<int32_t> vis(static_cast<size_t>(capacity));
-  const int nvis = oracle_visible_chunks(q_chunk, n_sink, window, capacity, vis.data());
-  if (nvis < 0) return -1;
   const double sigma = softmax_scale > 0.0 ? softmax_scale : 1.0 / std::sqrt(static_cast<double>(d));
   const int64_t T = static_cast<int64_t>(chunk_tokens) * capacity;
 
@@ -283,6 +301,47 @@ int oracle_attention_rows(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, i
     for (int32_t e = 0; e < d; ++e) out[static_cast<int64_t>(r) * d + e] = o[e] / denom;
   }
   return 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+int oracle_attention_rows(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, int32_t d,
+                          int64_t q_token_stride,
+                          const uint8_t* k_codes, const uint8_t* k_scales, const float* k_gscale,
+                          const uint8_t* v_codes, const uint8_t* v_scales, const float* v_gscale,
+                          int32_t chunk_tokens, int32_t capacity,
+                          int32_t q_chunk, int32_t n_sink, int32_t window, double softmax_scale,
+                          const int32_t* rows, int32_t n_rows, double* out) {
+  if (capacity <= 0) return -1;
+  std::vector<int32_t> vis(static_cast<size_t>(capacity));
+  const int nvis = oracle_visible_chunks(q_chunk, n_sink, window, capacity, vis.data());
+  if (nvis < 0) return -1;
+  return attention_over_slots(q, B, Lq, H, d, q_token_stride, k_codes, k_scales, k_gscale, v_codes,
+                              v_scales, v_gscale, chunk_tokens, capacity, vis.data(), nvis,
+                              softmax_scale, rows, n_rows, out);
+}
+
+int oracle_attention_rows_slots(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, int32_t d,
+                                int64_t q_token_stride,
+                                const uint8_t* k_codes, const uint8_t* k_scales, const float* k_gscale,
+                                const uint8_t* v_codes, const uint8_t* v_scales, const float* v_gscale,
+                                int32_t chunk_tokens, int32_t capacity, const int32_t* slots,
+                                int32_t n_slots, double softmax_scale, const int32_t* rows,
+                                int32_t n_rows, double* out) {
+  if (capacity <= 0 || !slots || n_slots < 1) return -1;
+  std::vector<char> listed(static_cast<size_t>(capacity), 0);  /* the union of the listed slots */
+  for (int32_t i = 0; i < n_slots; ++i) {
+    if (slots[i] < 0 || slots[i] >= capacity) return -1;
+    listed[static_cast<size_t>(slots[i])] = 1;
+  }
+  std::vector<int32_t> vis;
+  for (int32_t c = 0; c < capacity; ++c)
+    if (listed[static_cast<size_t>(c)]) vis.push_back(c);
+  return attention_over_slots(q, B, Lq, H, d, q_token_stride, k_codes, k_scales, k_gscale, v_codes,
+                              v_scales, v_gscale, chunk_tokens, capacity, vis.data(),
+                              static_cast<int>(vis.size()), softmax_scale, rows, n_rows, out);
 }
 
 }  // extern "C"

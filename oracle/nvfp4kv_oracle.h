@@ -66,6 +66,15 @@ int oracle_dequantize(const uint8_t* codes, const uint8_t* scales, const float* 
 int oracle_visible_chunks(int32_t q_chunk, int32_t n_sink, int32_t window, int32_t capacity,
                           int32_t* out);
 
+/* The effective chunk set of a multi-shot attention sink (paper page, section 4.2 "Inference with
+ * Multi-Shot Attention Sink"; reading note, "Multi-shot attention sinks"): the global sink
+ * {c < n_sink}, the current shot's sink {shot_start <= c < shot_start + shot_len} and the sliding
+ * window {q_chunk - window < c <= q_chunk}, overlaps counted once, ascending, clipped to
+ * [0, capacity); the shot sink must end at or before the query chunk (it is history).
+ * shot_len = 0 gives oracle_visible_chunks.  Returns the count or -1. */
+int oracle_multishot_chunks(int32_t q_chunk, int32_t n_sink, int32_t window, int32_t shot_start,
+                            int32_t shot_len, int32_t capacity, int32_t* out);
+
 /* fp64 attention of selected query rows over the dequantised cache.
  * q       : bf16 bit patterns, element (b, i, h, e) at q[(b*Lq + i)*q_token_stride + h*d + e]
  * rows    : n_rows triples (b, h, i)
@@ -78,6 +87,16 @@ int oracle_attention_rows(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, i
                           int32_t chunk_tokens, int32_t capacity,
                           int32_t q_chunk, int32_t n_sink, int32_t window, double softmax_scale,
                           const int32_t* rows, int32_t n_rows, double* out);
+
+/* The same attention over the keys of the listed chunk slots (any order; a slot listed twice counts
+ * once; each in [0, capacity); n_slots >= 1).  Returns 0 or -1 for bad arguments. */
+int oracle_attention_rows_slots(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, int32_t d,
+                                int64_t q_token_stride,
+                                const uint8_t* k_codes, const uint8_t* k_scales, const float* k_gscale,
+                                const uint8_t* v_codes, const uint8_t* v_scales, const float* v_gscale,
+                                int32_t chunk_tokens, int32_t capacity, const int32_t* slots,
+                                int32_t n_slots, double softmax_scale, const int32_t* rows,
+                                int32_t n_rows, double* out);
 
 #ifdef __cplusplus
 }
