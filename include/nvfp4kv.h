@@ -146,6 +146,20 @@ int nvfp4_kv_attention(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q
                        int32_t window_chunks, float softmax_scale, void* out, int32_t out_dtype,
                        void* workspace, size_t workspace_bytes, void* cuda_stream);
 
+/* Attention over an explicit set of visible chunk slots: the multi-shot sink of the paper page,
+ * section 4.2 "Inference with Multi-Shot Attention Sink", and the reading note, "Multi-shot
+ * attention sinks", where besides the global sink each shot keeps its own sink chunks.  The caller
+ * lists the slots (global sink, shot sinks, local window, in any order; repeats are counted once):
+ *     out_i = sum_j softmax_j(scale * q_i . k_hat_j) v_hat_j    over the keys j of the listed slots.
+ *   slots    host int32[n_slots], each in [0, capacity); n_slots >= 1
+ * The slots, sorted, may form at most 4 runs of consecutive slots (more gives
+ * NVFP4KV_ERR_UNSUPPORTED before anything is launched).  Other arguments, results and errors as
+ * for nvfp4_kv_attention, which is this call with the slots V(q_chunk) above. */
+int nvfp4_kv_attention_slots(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q_tokens,
+                             int64_t q_token_stride, const int32_t* slots, int32_t n_slots,
+                             float softmax_scale, void* out, int32_t out_dtype, void* workspace,
+                             size_t workspace_bytes, void* cuda_stream);
+
 /* Dequantise chunk slots [first_slot, first_slot + n_slots) of K (which == 0) or V
  * (which == 1) into device fp32 out[batch][heads][n_slots*chunk_tokens][head_dim]: the
  * pages' dequantisation step on its own, for tests and diagnostics.  Each value is the

@@ -48,6 +48,8 @@ SIGNATURES = {
     "nvfp4_kv_quantize_static_scratch": (ctypes.c_int, [_CP, _i32, _vp, _vp, _i64, _vp]),
     "nvfp4_kv_attention": (ctypes.c_int, [_CP, _vp, _i32, _i64, _i32, _i32, _i32, ctypes.c_float,
                                           _vp, _i32, _vp, _sz, _vp]),
+    "nvfp4_kv_attention_slots": (ctypes.c_int, [_CP, _vp, _i32, _i64, ctypes.POINTER(_i32), _i32,
+                                                ctypes.c_float, _vp, _i32, _vp, _sz, _vp]),
     "nvfp4_kv_dequantize": (ctypes.c_int, [_CP, _i32, _i32, _i32, _vp, _vp]),
     "nvfp4kv_debug_encode": (ctypes.c_int, [_vp, _i64, _vp, _vp, _vp]),
     "nvfp4kv_quantize_launches": (ctypes.c_int, [_CP]),
@@ -174,13 +176,9 @@ class KVCache:
             raise NvFp4KvError(-n, "nvfp4kv_quantize_launches")
         return n
 
-    def attention(self, q, q_chunk: int, n_sink: int, window: int, softmax_scale: float = 0.0,
-                  out=None, out_dtype=None, stream=None):
-        """Attention of bf16 queries ``q`` ([B, Lq, H, 128]) of chunk ``q_chunk`` over the
-        sink + window chunks of the cache.  Returns ``out`` ([B, Lq, H, 128], fp32 by default)."""
+    def _out_for(self, q, out, out_dtype):
         import torch
         Lq = q.shape[1]
-        qs = _token_stride(q, "q", Lq, self.heads)
         if out is None:
             out = torch.empty(q.shape[0], Lq, self.heads, HEAD_DIM,
                               dtype=torch.float32 if out_dtype is None else out_dtype, device=q.device)
@@ -189,12 +187,45 @@ class KVCache:
         code = {torch.float32: OUT_F32, torch.bfloat16: OUT_BF16}.get(out.dtype)
         if code is None:
             raise ValueError("out must be fp32 or bf16")
+        return out, code
+
+    def attention(self, q, q_chunk: int, n_sink: int, window: int, softmax_scale: float = 0.0,
+                  out=None, out_dtype=None, stream=None):
+        """Attention of bf16 queries ``q`` ([B, Lq, H, 128]) of chunk ``q_chunk`` over the
+        sink + window chunks of the cache.  Returns ``out`` ([B, Lq, H, 128], fp32 by default)."""
+        Lq = q.shape[1]
+        qs = _token_stride(q, "q", Lq, self.heads)
+        out, code = self._out_for(q, out, out_dtype)
         self.reserve_workspace(Lq)
         _check(lib().nvfp4_kv_attention(ctypes.byref(self.desc), q.data_ptr(), Lq, qs, q_chunk, n_sink,
                                         window, float(softmax_scale), out.data_ptr(), code,
                                         self._ws.data_ptr(), self._ws.numel(), _stream_handle(stream)),
                "nvfp4_kv_attention")
         return out
+
+    def attention_slots(self, q, slots, softmax_scale: float = 0.0, out=None, out_dtype=None,
+                        stream=None):
+        """Attention of ``q`` over the keys of the listed chunk slots (any order, repeats once)."""
+        Lq = q.shape[1]
+        qs = _token_stride(q, "q", Lq, self.heads)
+        out, code = self._out_for(q, out, out_dtype)
+        sl = (_i32 * max(len(slots), 1))(*[int(x) for x in slots])
+        self.reserve_workspace(Lq)
+        _check(lib().nvfp4_kv_attention_slots(ctypes.byref(self.desc), q.data_ptr(), Lq, qs, sl, len(slots),
+                                              float(softmax_scale), out.data_ptr(), code,
+                                              self._ws.data_ptr(), self._ws.numel(), _stream_handle(stream)),
+               "nvfp4_kv_attention_slots")
+        return out
+
+    def attention_multishot(self, q, q_chunk: int, n_sink: int, window: int, shot_start: int,
+                            shot_len: int, **kw):
+        """Multi-shot attention sink: global sink {c < n_sink}, the current shot's sink
+        {shot_start <= c < shot_start + shot_len} and the window {q_chunk - window < c <= q_chunk}."""
+        if shot_start < 0 or shot_len < 0 or shot_start + shot_len > q_chunk + 1:
+            raise ValueError("the shot sink must lie in [0, q_chunk]")
+        slots = sorted(set(range(min(n_sink, self.capacity))) | set(range(shot_start, shot_start + shot_len)) |
+                       set(range(max(0, q_chunk - window + 1), q_chunk + 1)))
+        return self.attention_slots(q, slots, **kw)
 
     def dequantize(self, which: str, first_slot: int = 0, n_slots: int | None = None, stream=None):
         """fp32 [B, H, n_slots*Lc, 128] dequantised K (``which='k'``) or V."""

@@ -2,6 +2,9 @@
 // workspace sizing and dispatch to the kernels.  No device memory is allocated here.
 #include <cstdio>
 
+#include <algorithm>
+#include <vector>
+
 #include "internal.h"
 
 using namespace nvfp4kv;
@@ -40,6 +43,33 @@ int check_device() {
     return NVFP4KV_ERR_CUDA;
   if (major != 10 || minor != 0) return NVFP4KV_ERR_UNSUPPORTED;
   return NVFP4KV_OK;
+}
+
+}  // namespace
+
+namespace {
+
+// Checks shared by both attention entry points, then the launch; vis is ascending and distinct.
+int attention_checked(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q_tokens,
+                      int64_t q_token_stride, const std::vector<int>& vis, float softmax_scale,
+                      void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                      void* cuda_stream) {
+  if (!q_bf16 || !out || !aligned16(q_bf16) || !aligned16(out)) return NVFP4KV_ERR_INVALID_ARG;
+  if (q_tokens <= 0 || q_tokens > (1 << 24)) return NVFP4KV_ERR_INVALID_ARG;
+  if (q_token_stride < static_cast<int64_t>(cache->heads) * cache->head_dim || q_token_stride % 8 != 0)
+    return NVFP4KV_ERR_INVALID_ARG;
+  if (out_dtype != NVFP4KV_OUT_F32 && out_dtype != NVFP4KV_OUT_BF16) return NVFP4KV_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale)) return NVFP4KV_ERR_INVALID_ARG;  // NaN
+  if (vis.empty()) return NVFP4KV_ERR_INVALID_ARG;
+  if (attention_runs(vis) > kAttnMaxRuns) return NVFP4KV_ERR_UNSUPPORTED;
+  const size_t need = attention_workspace_bytes(*cache, q_tokens);
+  if (need > 0 && (!workspace || !aligned16(workspace) || workspace_bytes < need))
+    return NVFP4KV_ERR_WORKSPACE;
+  const int rc = check_device();
+  if (rc != NVFP4KV_OK) return rc;
+  return launch_attention(*cache, static_cast<const uint16_t*>(q_bf16), q_tokens, q_token_stride, vis,
+                          softmax_scale, out, out_dtype, workspace, workspace_bytes,
+                          static_cast<cudaStream_t>(cuda_stream));
 }
 
 }  // namespace
@@ -115,22 +145,33 @@ int nvfp4_kv_attention(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q
                        void* workspace, size_t workspace_bytes, void* cuda_stream) {
   int rc = check_cache(cache);
   if (rc != NVFP4KV_OK) return rc;
-  if (!q_bf16 || !out || !aligned16(q_bf16) || !aligned16(out)) return NVFP4KV_ERR_INVALID_ARG;
-  if (q_tokens <= 0 || q_tokens > (1 << 24)) return NVFP4KV_ERR_INVALID_ARG;
-  if (q_token_stride < static_cast<int64_t>(cache->heads) * cache->head_dim || q_token_stride % 8 != 0)
-    return NVFP4KV_ERR_INVALID_ARG;
   if (q_chunk < 0 || q_chunk >= cache->capacity_chunks || n_sink_chunks < 0 || window_chunks < 1)
     return NVFP4KV_ERR_INVALID_ARG;
-  if (out_dtype != NVFP4KV_OUT_F32 && out_dtype != NVFP4KV_OUT_BF16) return NVFP4KV_ERR_INVALID_ARG;
-  if (!(softmax_scale == softmax_scale)) return NVFP4KV_ERR_INVALID_ARG;  // NaN
-  const size_t need = attention_workspace_bytes(*cache, q_tokens);
-  if (need > 0 && (!workspace || !aligned16(workspace) || workspace_bytes < need))
-    return NVFP4KV_ERR_WORKSPACE;
-  rc = check_device();
+  // V(t) = {c < n_sink} U {t - window < c <= t}, each slot once, ascending.
+  std::vector<int> vis;
+  for (int ch = 0; ch < cache->capacity_chunks; ++ch)
+    if (ch < n_sink_chunks || (ch > q_chunk - window_chunks && ch <= q_chunk)) vis.push_back(ch);
+  return attention_checked(cache, q_bf16, q_tokens, q_token_stride, vis, softmax_scale, out, out_dtype,
+                           workspace, workspace_bytes, cuda_stream);
+}
+
+int nvfp4_kv_attention_slots(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q_tokens,
+                             int64_t q_token_stride, const int32_t* slots, int32_t n_slots,
+                             float softmax_scale, void* out, int32_t out_dtype, void* workspace,
+                             size_t workspace_bytes, void* cuda_stream) {
+  int rc = check_cache(cache);
   if (rc != NVFP4KV_OK) return rc;
-  return launch_attention(*cache, static_cast<const uint16_t*>(q_bf16), q_tokens, q_token_stride,
-                          q_chunk, n_sink_chunks, window_chunks, softmax_scale, out, out_dtype,
-                          workspace, workspace_bytes, static_cast<cudaStream_t>(cuda_stream));
+  if (!slots || n_slots < 1) return NVFP4KV_ERR_INVALID_ARG;
+  std::vector<int> vis;
+  vis.reserve(static_cast<size_t>(n_slots));
+  for (int32_t i = 0; i < n_slots; ++i) {
+    if (slots[i] < 0 || slots[i] >= cache->capacity_chunks) return NVFP4KV_ERR_INVALID_ARG;
+    vis.push_back(slots[i]);
+  }
+  std::sort(vis.begin(), vis.end());  // the union of the listed chunks, each once
+  vis.erase(std::unique(vis.begin(), vis.end()), vis.end());
+  return attention_checked(cache, q_bf16, q_tokens, q_token_stride, vis, softmax_scale, out, out_dtype,
+                           workspace, workspace_bytes, cuda_stream);
 }
 
 int nvfp4_kv_dequantize(const nvfp4kv_cache* cache, int32_t which, int32_t first_slot,

@@ -57,7 +57,7 @@ constexpr int PK_CODES = BN * kCodeBytes;               // 8192
 constexpr int PK_BYTES = PK_CODES + BN * kScaleBytes;   // 9216
 constexpr int TILE16 = BN * D * 2;                      // one 128 x 128 16-bit operand tile
 constexpr int HALF16 = TILE16 / 2;                      // 128 rows x 64 elements (128 B rows)
-constexpr int MAX_RUNS = 4;
+constexpr int MAX_RUNS = kAttnMaxRuns;
 
 template <int QT>
 struct Cfg {
@@ -843,9 +843,16 @@ int attention_plan(const nvfp4kv_cache& c, int q_tokens, int n_sms, int cta, int
   return NVFP4KV_OK;
 }
 
+int attention_runs(const std::vector<int>& vis) {
+  int runs = 0;
+  for (size_t i = 0; i < vis.size(); ++i)
+    if (i == 0 || vis[i] != vis[i - 1] + 1) ++runs;
+  return runs;
+}
+
 int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, int64_t q_stride,
-                     int q_chunk, int n_sink, int window, float softmax_scale, void* out,
-                     int out_dtype, void*, size_t, cudaStream_t stream) {
+                     const std::vector<int>& vis, float softmax_scale, void* out, int out_dtype, void*,
+                     size_t, cudaStream_t stream) {
   AttnParams prm{};
   prm.k_codes = c.k_codes;
   prm.v_codes = c.v_codes;
@@ -865,11 +872,8 @@ int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, in
   const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(D));
   prm.scale_log2 = scale * 1.4426950408889634f;
 
-  // Visible chunk slots {c < n_sink} U {q_chunk - window < c <= q_chunk}, merged into runs of
-  // consecutive slots; KV tiles never cross a run boundary.
-  std::vector<int> vis;
-  for (int ch = 0; ch < c.capacity_chunks; ++ch)
-    if (ch < n_sink || (ch > q_chunk - window && ch <= q_chunk)) vis.push_back(ch);
+  // The visible chunk slots (ascending, distinct), merged into runs of consecutive slots; KV
+  // tiles never cross a run boundary.
   prm.n_runs = 0;
   prm.run_tile0[0] = 0;
   for (size_t i = 0; i < vis.size();) {

@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <vector>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -37,13 +38,17 @@ int quantize_launches(const nvfp4kv_cache& c);
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // ---- attention (attention.cu)
+constexpr int kAttnMaxRuns = 4;  // runs of consecutive visible chunk slots one attention call takes
 size_t attention_workspace_bytes(const nvfp4kv_cache& c, int q_tokens);
+// Number of runs of consecutive slots in an ascending, duplicate-free slot list.
+int attention_runs(const std::vector<int>& vis);
 // The attention launch's work split for n_sms SMs: out[0] = CTAs; for cta >= 0 also its work item
 // out[1] = batch * heads + head index, out[2] = first query row, out[3] = query tiles (1 or 2).
 int attention_plan(const nvfp4kv_cache& c, int q_tokens, int n_sms, int cta, int out[4]);
+// vis: the visible chunk slots, ascending and distinct, at most kAttnMaxRuns runs.
 int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, int64_t q_stride,
-                     int q_chunk, int n_sink, int window, float softmax_scale, void* out,
-                     int out_dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+                     const std::vector<int>& vis, float softmax_scale, void* out, int out_dtype,
+                     void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 // ---- diagnostics (dequantize.cu)
 cudaError_t launch_dequantize(const nvfp4kv_cache& c, int which, int first_slot, int n_slots,

@@ -71,6 +71,21 @@ def _attn(L, d, q=0x80000, lq=64, stride=256, q_chunk=3, sink=1, window=3, out=0
                                 dtype, ws, ws_bytes, None)
 
 
+def _attn_slots(L, d, slots, q=0x80000, lq=64, stride=256, out=0x90000, dtype=0):
+    arr = (ctypes.c_int32 * max(len(slots), 1))(*slots)
+    return L.nvfp4_kv_attention_slots(ctypes.byref(d), q, lq, stride, arr if slots else None, len(slots),
+                                      0.0, out, dtype, 0xA0000, 1 << 20, None)
+
+
+def test_attention_slot_list_argument_checks(L):
+    d = _desc(capacity_chunks=12)
+    assert _attn_slots(L, d, []) == nk.ERR_INVALID_ARG
+    assert _attn_slots(L, d, [0, 12]) == nk.ERR_INVALID_ARG        # slot >= capacity
+    assert _attn_slots(L, d, [-1]) == nk.ERR_INVALID_ARG
+    assert _attn_slots(L, d, [0, 2, 4, 6, 8]) == nk.ERR_UNSUPPORTED  # five runs of slots
+    assert _attn_slots(L, d, [0, 2, 4, 6, 7], lq=0) == nk.ERR_INVALID_ARG
+
+
 def test_quantize_argument_checks(L):
     assert L.nvfp4_kv_quantize(None, 0, 0x80000, 0x90000, 256, 0xA0000, 1 << 20, None) == nk.ERR_INVALID_ARG
     assert _quant(L, _desc(head_dim=64)) == nk.ERR_UNSUPPORTED
@@ -117,6 +132,8 @@ def test_valid_arguments_without_a_gpu_report_a_cuda_error(L):
         pytest.skip("a GPU is present")
     assert _quant(L, _desc()) == nk.ERR_CUDA
     assert _attn(L, _desc()) == nk.ERR_CUDA
+    # four runs, listed out of order and with repeats: valid, so it reaches the device check
+    assert _attn_slots(L, _desc(capacity_chunks=12), [9, 0, 4, 5, 0, 7, 9]) == nk.ERR_CUDA
     assert L.nvfp4kv_quantize_launches(ctypes.byref(_desc())) == -nk.ERR_CUDA
 
 

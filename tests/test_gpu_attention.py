@@ -143,3 +143,53 @@ def test_queries_beyond_fp16_range_use_an_exact_power_of_two_prescale():
                      for i in range(w.q_tokens)], np.int32)
     want = oracle.attention_rows(qb, ocache, w.q_chunk, w.n_sink, w.window, rows)
     assert_attention_close(gather_rows(out.cpu().numpy(), rows), want, "large q")
+
+
+# ---- multi-shot attention sink (paper page, section 4.2; reading note, "Multi-shot attention
+# sinks"): global sink U the current shot's sink U window, through the slot-list entry point.
+MS = dataclasses.replace(W["tiny"], key="multishot", batch=1, heads=2, chunk_tokens=64, capacity=12,
+                         q_chunk=9, n_sink=1, window=2, q_tokens=100)
+
+
+def _ms_case(slots_listed, layer=0):
+    w = MS
+    vis = sorted(set(slots_listed))
+    cache, ocache = make_caches(w, vis, layer)
+    qb = synthetic.queries(w, layer)
+    out = cache.attention_slots(dev_bf16(qb), slots_listed)
+    assert cache.read_status() == 0
+    rows = np.array([(b, h, i) for b in range(w.batch) for h in range(w.heads)
+                     for i in range(w.q_tokens)], np.int32)
+    want = oracle.attention_rows_slots(qb, ocache, slots_listed, rows)
+    return gather_rows(out.float().cpu().numpy(), rows), want, cache, qb
+
+
+def test_multishot_sink_three_runs_all_rows():
+    # global sink {0}, shot sink (start 4, length 2), window {8, 9}: runs [0], [4, 5], [8, 9]
+    slots = oracle.multishot_chunks(9, 1, 2, 4, 2, MS.capacity)
+    assert slots == [0, 4, 5, 8, 9]
+    got, want, *_ = _ms_case(slots)
+    assert_attention_close(got, want, "multishot 3 runs")
+
+
+def test_slot_list_four_runs_out_of_order_with_repeats():
+    got, want, *_ = _ms_case([9, 0, 3, 6, 7, 3, 9, 0])
+    assert_attention_close(got, want, "slot list 4 runs")
+
+
+def test_multishot_binding_matches_the_oracle_set():
+    import torch
+    _, _, cache, qb = _ms_case(oracle.multishot_chunks(9, 1, 2, 4, 2, MS.capacity))
+    a = cache.attention_multishot(dev_bf16(qb), 9, 1, 2, 4, 2)
+    b = cache.attention_slots(dev_bf16(qb), [0, 4, 5, 8, 9])
+    assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
+def test_window_slot_list_equals_the_window_call_bit_for_bit():
+    import torch
+    w = dataclasses.replace(W["tiny"], **EDGE["ragged_two_runs"])
+    cache, _ = make_caches(w, w.visible_chunks)
+    q = dev_bf16(synthetic.queries(w))
+    a = cache.attention(q, w.q_chunk, w.n_sink, w.window)
+    b = cache.attention_slots(q, list(reversed(w.visible_chunks)))
+    assert torch.equal(a.view(torch.int32), b.view(torch.int32))
