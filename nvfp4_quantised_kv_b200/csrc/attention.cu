@@ -35,9 +35,9 @@
 
 #include <algorithm>
 #include <cmath>
-#include <functional>
+#include <map>
 #include <mutex>
-#include <queue>
+#include <tuple>
 #include <vector>
 
 #include "internal.h"
@@ -766,47 +766,65 @@ cudaError_t launch(const CUtensorMap& tm, const AttnParams& prm, int n_single_ct
   return cudaGetLastError();
 }
 
-// Makespan, in units of one two-tile CTA, of p two-tile and s one-tile CTAs dealt in launch order
-// to g SMs (one CTA per SM at a time), a one-tile CTA costing `single` of a two-tile one.
-double makespan(int p, int s, int g, double single) {
-  std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
-  for (int i = 0; i < g; ++i) free_at.push(0.0);
-  double end = 0.0;
-  for (int i = 0; i < p + s; ++i) {
-    const double t = free_at.top() + (i < p ? 1.0 : single);
-    free_at.pop();
-    free_at.push(t);
-    end = std::max(end, t);
+// Makespan of p two-tile CTAs (cost `pair`) followed by s one-tile CTAs (cost `single`), each
+// started on whichever of the g SMs frees first (one CTA per SM at a time).  Integer costs keep
+// equal loads equal; machines are tracked per load level, so the cost is the number of levels the
+// schedule passes through, not the number of CTAs.
+int64_t makespan(int64_t p, int64_t s, int64_t g, int64_t pair, int64_t single) {
+  std::map<int64_t, int64_t> level;  // load -> machines at that load
+  level[(p / g) * pair] += g - p % g;
+  if (p % g) level[(p / g + 1) * pair] += p % g;
+  while (s > 0) {
+    auto lo = level.begin();
+    const int64_t take = std::min(lo->second, s);
+    const int64_t load = lo->first;
+    s -= take;
+    if ((lo->second -= take) == 0) level.erase(lo);
+    level[load + single] += take;
   }
-  return end;
+  return level.rbegin()->first;
 }
 
 // Splits the n_qt query tiles of each of the bh (batch, head) pairs into tile pairs (two-tile CTAs,
 // the two softmax warpgroups in ping-pong) and single tiles (one-tile CTAs) so that the launch
 // finishes soonest on g SMs: e.g. 444 tiles on 148 SMs as 148 pairs + 148 singles (1.94 units)
-// instead of 222 pairs in two waves (2 units).  Candidates: all pairs, no pairs, whole waves of
-// pairs.
+// instead of 222 pairs in two waves (2 units).  Candidates: all pairs, no pairs, and the last
+// three whole waves of pairs.  Plans are cached per (n_qt, bh, g).
 void plan_work(int n_qt, int bh, int g, AttnParams& prm, int& n_single_ctas) {
-  // Cost of a one-tile CTA relative to a two-tile one, measured on the 1.3B-class layer: the
-  // per-KV-tile dequantisation and MMA chain, which do not shrink with one query tile, dominate.
-  constexpr double kSingle = 0.94;
-  const int max_p = bh * (n_qt / 2), total = bh * n_qt;
-  std::vector<int> cand = {0, max_p};
-  for (int k = 1; k * g <= max_p; ++k) cand.push_back(k * g);
-  int best_p = max_p;
-  double best = makespan(max_p, total - 2 * max_p, g, kSingle);
-  for (int pc : cand) {
-    const double m = makespan(pc, total - 2 * pc, g, kSingle);
-    if (m < best - 1e-9 || (m < best + 1e-9 && pc > best_p)) {
-      best = m;
-      best_p = pc;
+  // Cost of a one-tile CTA relative to a two-tile one (94 : 100), measured on the 1.3B-class
+  // layer: the per-KV-tile dequantisation and MMA chain, which do not shrink with one query tile,
+  // dominate.
+  constexpr int64_t kPair = 100, kSingle = 94;
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int>, int> cache;
+  int best_p = -1;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(std::make_tuple(n_qt, bh, g));
+    if (it != cache.end()) best_p = it->second;
+  }
+  const int64_t max_p = static_cast<int64_t>(bh) * (n_qt / 2), total = static_cast<int64_t>(bh) * n_qt;
+  if (best_p < 0) {
+    std::vector<int64_t> cand = {0, max_p};
+    for (int64_t k = max_p / g; k >= 1 && k >= max_p / g - 2; --k) cand.push_back(k * g);
+    int64_t bp = max_p, best = makespan(max_p, total - 2 * max_p, g, kPair, kSingle);
+    for (int64_t pc : cand) {
+      const int64_t m = makespan(pc, total - 2 * pc, g, kPair, kSingle);
+      if (m < best || (m == best && pc > bp)) {
+        best = m;
+        bp = pc;
+      }
     }
+    best_p = static_cast<int>(bp);
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache.size() > 4096) cache.clear();
+    cache[std::make_tuple(n_qt, bh, g)] = best_p;
   }
   prm.n_qt = n_qt;
   prm.pp = best_p / bh;
   prm.pr = best_p % bh;
   prm.n_pair_ctas = best_p;
-  n_single_ctas = total - 2 * best_p;
+  n_single_ctas = static_cast<int>(total - 2 * best_p);
 }
 
 }  // namespace

@@ -60,3 +60,19 @@ def test_plan_argument_checks(L):
     assert _plan(L, d, 64, 148, 99)[0] == nk.ERR_INVALID_ARG
     assert L.nvfp4kv_attention_plan(ctypes.byref(d), 64, 148, -1, None) == nk.ERR_INVALID_ARG
     assert L.nvfp4kv_attention_plan(None, 64, 148, -1, (ctypes.c_int32 * 4)()) == nk.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("lq,heads,pairs", [(4680, 12, 148), (2640, 24, 240), (880, 24, 72)])
+def test_benchmarked_shapes_plan_as_documented(L, lq, heads, pairs):
+    d = _desc(batch=1, heads=heads)
+    n = _plan(L, d, lq, 148, -1)[1][0]
+    assert sum(_plan(L, d, lq, 148, c)[1][3] == 2 for c in range(n)) == pairs
+
+
+def test_planning_a_very_large_launch_is_cheap(L):
+    import time
+    d = _desc(batch=64, heads=64)
+    t0 = time.perf_counter()
+    rc, out = _plan(L, d, 16384 + 77, 148, -1)  # 64*64 heads x 129 query tiles
+    assert rc == nk.OK and out[0] > 0
+    assert time.perf_counter() - t0 < 0.5
