@@ -330,8 +330,14 @@ def main():
     traffic = None
     prof = os.path.join(ROOT, "profiles", f"traffic_{w.key}.json")
     if os.path.exists(prof):
+        # the DRAM bytes of one ncu capture, valid only for the attention source they were taken on
+        import hashlib
         with open(prof) as f:
-            traffic = json.load(f).get("attention_dram_bytes_per_launch")
+            rec = json.load(f)
+        with open(os.path.join(ROOT, "nvfp4_quantised_kv_b200", "csrc", "attention.cu"), "rb") as f:
+            src_sha = hashlib.sha256(f.read()).hexdigest()
+        if rec.get("attention_cu_sha256") == src_sha:
+            traffic = rec.get("attention_dram_bytes_per_launch")
 
     if rank == 0:
         line = {
