@@ -192,6 +192,13 @@ int nvfp4kv_attention_plan(const nvfp4kv_cache* cache, int32_t q_tokens, int32_t
  * the pages; a negative result is minus an nvfp4kv_status code (invalid cache, no sm_100 device). */
 int nvfp4kv_quantize_launches(const nvfp4kv_cache* cache);
 
+/* Fault injection for tests of the failure path, no counterpart in the pages: launches a one-warp
+ * kernel whose bounded wait is made to run out (nothing ever arrives at its barrier).  After the
+ * kernels' wait limit (about 1 s) it ORs 1 << NVFP4KV_ERR_DEVICE_TIMEOUT into the cache's status
+ * word and returns; the CUDA context stays usable.  No GPU fault, trap or hang is involved.
+ * Errors: NVFP4KV_ERR_INVALID_ARG (bad cache), NVFP4KV_ERR_UNSUPPORTED, NVFP4KV_ERR_CUDA. */
+int nvfp4kv_debug_wait_timeout(const nvfp4kv_cache* cache, void* cuda_stream);
+
 /* Wait for `cuda_stream`, then read the cache's device status word into *out and clear it.
  * *out == 0 means no device-side error since the last read; otherwise it holds OR-ed
  * nvfp4kv_status bits (1 << NVFP4KV_ERR_DEVICE_TIMEOUT for a bounded wait that ran out). */

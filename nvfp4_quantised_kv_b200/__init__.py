@@ -54,6 +54,7 @@ SIGNATURES = {
     "nvfp4kv_debug_encode": (ctypes.c_int, [_vp, _i64, _vp, _vp, _vp]),
     "nvfp4kv_quantize_launches": (ctypes.c_int, [_CP]),
     "nvfp4kv_attention_plan": (ctypes.c_int, [_CP, _i32, _i32, _i32, ctypes.POINTER(_i32)]),
+    "nvfp4kv_debug_wait_timeout": (ctypes.c_int, [_CP, _vp]),
     "nvfp4kv_read_status": (ctypes.c_int, [_CP, _vp, ctypes.POINTER(ctypes.c_uint32)]),
     "nvfp4kv_strerror": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -168,6 +169,11 @@ class KVCache:
         _check(lib().nvfp4_kv_quantize(ctypes.byref(self.desc), slot, k.data_ptr(), v.data_ptr(), ks,
                                        self._ws.data_ptr(), self._ws.numel(), _stream_handle(stream)),
                "nvfp4_kv_quantize")
+
+    def debug_wait_timeout(self, stream=None) -> None:
+        """Fault injection: a kernel whose bounded wait runs out sets the device-timeout bit."""
+        _check(lib().nvfp4kv_debug_wait_timeout(ctypes.byref(self.desc), _stream_handle(stream)),
+               "nvfp4kv_debug_wait_timeout")
 
     def quantize_launches(self) -> int:
         """Kernels one ``quantize`` call launches for this cache on the current device (1 or 2)."""

@@ -199,6 +199,16 @@ int nvfp4kv_debug_encode(const float* x, int64_t n, uint8_t* e2m1_codes, uint8_t
   return e == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 
+int nvfp4kv_debug_wait_timeout(const nvfp4kv_cache* cache, void* cuda_stream) {
+  const int rc = check_cache(cache);
+  if (rc != NVFP4KV_OK) return rc;
+  const int dc = check_device();
+  if (dc != NVFP4KV_OK) return dc;
+  return launch_wait_timeout_probe(cache->status, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess
+             ? NVFP4KV_OK
+             : NVFP4KV_ERR_CUDA;
+}
+
 int nvfp4kv_attention_plan(const nvfp4kv_cache* cache, int32_t q_tokens, int32_t n_sms, int32_t cta,
                            int32_t* out) {
   int rc = check_cache(cache);

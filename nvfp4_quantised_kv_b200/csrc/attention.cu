@@ -751,6 +751,21 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
   }
 }
 
+// Fault-injection probe: one warp waits, with the same bounded warp-collective wait the kernels
+// use, on an mbarrier that nothing arrives at.  After kWaitLimitNs the wait gives up, ORs
+// NVFP4KV_ERR_DEVICE_TIMEOUT into *status, and the kernel returns with the context intact.
+__global__ void __launch_bounds__(32) wait_timeout_probe(uint32_t* status) {
+  __shared__ __align__(8) uint64_t never_arrived;
+  __shared__ uint32_t abort_word;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(ptx::smem_u32(&never_arrived), 1);
+    abort_word = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncwarp();
+  waitw(ptx::smem_u32(&never_arrived), 0, &abort_word, status);
+}
+
 // ------------------------------------------------------------------ host side
 template <int QT>
 cudaError_t launch(const CUtensorMap& tm, const AttnParams& prm, int n_single_ctas, cudaStream_t stream) {
@@ -844,6 +859,11 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 size_t attention_workspace_bytes(const nvfp4kv_cache&, int) { return 0; }
+
+cudaError_t launch_wait_timeout_probe(uint32_t* status, cudaStream_t stream) {
+  wait_timeout_probe<<<1, 32, 0, stream>>>(status);
+  return cudaGetLastError();
+}
 
 int attention_plan(const nvfp4kv_cache& c, int q_tokens, int n_sms, int cta, int out[4]) {
   AttnParams prm{};

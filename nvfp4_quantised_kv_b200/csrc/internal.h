@@ -50,6 +50,10 @@ int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, in
                      const std::vector<int>& vis, float softmax_scale, void* out, int out_dtype,
                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+// A kernel whose bounded wait runs out (nothing arrives at its barrier): the device-timeout path,
+// for tests (attention.cu).
+cudaError_t launch_wait_timeout_probe(uint32_t* status, cudaStream_t stream);
+
 // ---- diagnostics (dequantize.cu)
 cudaError_t launch_dequantize(const nvfp4kv_cache& c, int which, int first_slot, int n_slots,
                               float* out, cudaStream_t stream);

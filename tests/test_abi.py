@@ -120,6 +120,7 @@ def test_dequantize_and_status_argument_checks(L):
     assert L.nvfp4_kv_dequantize(ctypes.byref(d), 0, 0, 1, 0x90008, None) == nk.ERR_INVALID_ARG
     assert L.nvfp4kv_read_status(None, None, None) == nk.ERR_INVALID_ARG
     assert L.nvfp4kv_quantize_launches(None) == -nk.ERR_INVALID_ARG
+    assert L.nvfp4kv_debug_wait_timeout(None, None) == nk.ERR_INVALID_ARG
     assert L.nvfp4kv_quantize_launches(ctypes.byref(_desc(head_dim=256))) == -nk.ERR_UNSUPPORTED
     assert L.nvfp4kv_debug_encode(None, 4, 0x1000, 0x2000, None) == nk.ERR_INVALID_ARG
     assert L.nvfp4kv_workspace_bytes(None, 64) == 0
@@ -135,6 +136,7 @@ def test_valid_arguments_without_a_gpu_report_a_cuda_error(L):
     # four runs, listed out of order and with repeats: valid, so it reaches the device check
     assert _attn_slots(L, _desc(capacity_chunks=12), [9, 0, 4, 5, 0, 7, 9]) == nk.ERR_CUDA
     assert L.nvfp4kv_quantize_launches(ctypes.byref(_desc())) == -nk.ERR_CUDA
+    assert L.nvfp4kv_debug_wait_timeout(ctypes.byref(_desc()), None) == nk.ERR_CUDA
 
 
 def test_strerror_covers_every_code(L):

@@ -111,6 +111,22 @@ def test_output_is_deterministic_and_bf16_output_is_rounded_fp32():
     assert torch.equal(ob.view(torch.int16), out.to(torch.bfloat16).view(torch.int16))
 
 
+def test_output_guard_rows_stay_untouched():
+    # the output lives between two guard batches filled with a canary pattern
+    import torch
+    w = dataclasses.replace(W["tiny"], **EDGE["ragged_two_runs"])
+    cache, _ = make_caches(w, w.visible_chunks)
+    q = dev_bf16(synthetic.queries(w))
+    big = torch.empty(w.batch + 2, w.q_tokens, w.heads, 128, dtype=torch.float32, device="cuda")
+    big.view(torch.int32).fill_(0x7FC0DEAD)
+    out = big[1:w.batch + 1]
+    cache.attention(q, w.q_chunk, w.n_sink, w.window, out=out)
+    assert cache.read_status() == 0
+    guard = torch.cat([big[0], big[w.batch + 1]]).view(torch.int32)
+    assert bool((guard == 0x7FC0DEAD).all())
+    assert bool(torch.isfinite(out).all())
+
+
 def test_query_token_stride_and_softmax_scale():
     import torch
     w = dataclasses.replace(W["tiny"], batch=2, heads=3)
