@@ -14,7 +14,8 @@
  *    E2M1 elements, one E4M3 scale per 16 elements (largest magnitudes 6 and 448), one FP32
  *    scale on top; dequantisation is the product of the three;
  *  - paper section 4.2 "Inference with Multi-Shot Attention Sink": sliding-window attention
- *    over a KV cache of W chunks plus a permanent global sink, overlaps deduplicated;
+ *    over a KV cache of W chunks plus a permanent global sink and, for multi-shot video, the
+ *    current shot's sink, overlaps deduplicated;
  *    section 2.1: a chunk attends to the preceding clean chunks and to its own tokens.
  *
  * Quantisation of one (chunk, head, tensor) with X = chunk_tokens x head_dim bf16 values,
@@ -27,8 +28,9 @@
  *
  * CONVENTIONS (all entry points)
  *  - Every pointer named "device" is CUDA device memory owned by the caller; the library
- *    never allocates, frees or keeps device memory, and keeps no state between calls other
- *    than a per-process cache of driver entry points.
+ *    never allocates or frees device memory.  It keeps no state between calls other than
+ *    per-process caches (driver entry points, per-shape launch plans and occupancy answers)
+ *    and the fixed 64 KiB scratch array of nvfp4_kv_quantize_static_scratch.
  *  - Calls are asynchronous on the given CUDA stream (a cudaStream_t passed as void*, NULL
  *    means the legacy default stream).  The return value reports host-side argument checks
  *    and launch errors only.  Errors found on the device (a bounded wait that ran out) are
