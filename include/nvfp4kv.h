@@ -89,12 +89,18 @@ int nvfp4kv_cache_sizes(int32_t batch, int32_t heads, int32_t head_dim, int32_t 
                         int32_t capacity_chunks, size_t* codes_bytes, size_t* scales_bytes,
                         size_t* gscale_bytes);
 
-/* Workspace bytes nvfp4_kv_quantize and nvfp4_kv_attention need for this cache and a query
- * chunk of q_tokens tokens (the maximum over both calls; 0 is never returned).  Returns 0
- * for an invalid cache description. */
+/* Workspace bytes nvfp4_kv_quantize and the attention calls need for this cache and a query
+ * chunk of q_tokens tokens (the maximum over the calls; 0 is never returned).  The attention
+ * part holds the partial results of work items split between CTAs: two slots of about 130 KB
+ * per SM of the CURRENT device (148 SMs are assumed when no device can be queried), so call it
+ * with the device that will run the attention current.  Returns 0 for an invalid cache
+ * description. */
 size_t nvfp4kv_workspace_bytes(const nvfp4kv_cache* cache, int32_t q_tokens);
 
-/* Quantise a new frame chunk's K and V and write it into chunk slot `chunk_slot`.
+/* Quantise a new frame chunk's K and V and write it into chunk slot `chunk_slot`: the
+ * re-quantisation of each new frame chunk's K and V into the NVFP4 cache (reading note,
+ * "The inference infrastructure"), in the three-level format of the reading note, "The NVFP4
+ * quantization format", and paper page section 2.2 (constants 16, 448, 6).
  *   k_bf16, v_bf16  device bf16, element (b, t, h, e) at [(b*chunk_tokens + t)*token_stride +
  *                   h*head_dim + e]; 16-byte aligned; token_stride >= heads*head_dim and a
  *                   multiple of 8
@@ -110,6 +116,30 @@ int nvfp4_kv_quantize(const nvfp4kv_cache* cache, int32_t chunk_slot, const void
                       const void* v_bf16, int64_t token_stride, void* workspace,
                       size_t workspace_bytes, void* cuda_stream);
 
+/* nvfp4_kv_quantize for the same new chunk slot of several layers' caches in one launch (the
+ * per-layer K and V of one generated frame chunk, as the reading note's "The inference
+ * infrastructure" re-quantises them).  Results are bit-identical to one nvfp4_kv_quantize call
+ * per layer.  The input crosses HBM once: a CTA reduces the maximum of one 128-token part of a
+ * (layer, tensor, b, h) slice, and encodes an earlier part once that part's slice is complete,
+ * re-reading rows that are still in L2.
+ *   caches         host array of n_layers cache descriptors, 1 <= n_layers <= 64, all with the
+ *                  same batch, heads, chunk_tokens and capacity
+ *   k_bf16, v_bf16 host arrays of n_layers device pointers, each laid out as for
+ *                  nvfp4_kv_quantize with the common token_stride
+ *   workspace      device scratch of at least nvfp4kv_quantize_layers_workspace_bytes() bytes;
+ *                  the call zeroes the counters it keeps there (a memset on the stream), so its
+ *                  contents on entry do not matter
+ * A device wait that runs out sets the timeout bit in caches[0]'s status word.  Errors as for
+ * nvfp4_kv_quantize; NVFP4KV_ERR_INVALID_ARG also for caches of different shapes and
+ * NVFP4KV_ERR_UNSUPPORTED for more than 64 layers or more than 2^31 parts. */
+int nvfp4_kv_quantize_layers(const nvfp4kv_cache* caches, int32_t n_layers, int32_t chunk_slot,
+                             const void* const* k_bf16, const void* const* v_bf16, int64_t token_stride,
+                             void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* Workspace bytes of nvfp4_kv_quantize_layers for n_layers caches shaped like caches[0]
+ * (0 for an invalid description). */
+size_t nvfp4kv_quantize_layers_workspace_bytes(const nvfp4kv_cache* caches, int32_t n_layers);
+
 /* nvfp4_kv_quantize without a workspace, for callers that cannot allocate device memory
  * (a pre-planned arena sized before this library was linked, a host framework that owns
  * every device allocation, a real-time loop that must not allocate).  The pages have no
@@ -122,15 +152,18 @@ int nvfp4_kv_quantize(const nvfp4kv_cache* cache, int32_t chunk_slot, const void
  *    nvfp4_kv_quantize for them.
  *  - The first call on each device looks up the array's device address (with that device
  *    current), which may load the library's GPU code: make that first call before any
- *    stream capture.
+ *    stream capture.  The address is kept until the process exits; resetting a device
+ *    (cudaDeviceReset) while the library is loaded is not supported by this entry point.
  *  - All calls share the one array and every call overwrites what it reads, so nothing needs
  *    clearing between calls; calls that may overlap on the GPU (unordered streams) race. */
 int nvfp4_kv_quantize_static_scratch(const nvfp4kv_cache* cache, int32_t chunk_slot,
                                      const void* k_bf16, const void* v_bf16, int64_t token_stride,
                                      void* cuda_stream);
 
-/* Attention of a chunk of bf16 queries over the NVFP4 cache.  The query chunk `q_chunk`
- * attends to the keys of the visible chunk slots
+/* Attention of a chunk of bf16 queries over the NVFP4 cache, dequantised inside the kernel
+ * (paper page, section 1 and section 3.2 "Parallel KV Quantization"), with the sliding window
+ * and permanent sink of paper page section 4.2 and the chunk's own tokens (section 2.1).  The
+ * query chunk `q_chunk` attends to the keys of the visible chunk slots
  *     V = { c < n_sink_chunks } U { q_chunk - window_chunks < c <= q_chunk },
  * each slot once (its own chunk included, so it must have been quantised first):
  *     out_i = sum_j softmax_j(scale * q_i . k_hat_j) v_hat_j    over the keys j of V.
@@ -140,8 +173,10 @@ int nvfp4_kv_quantize_static_scratch(const nvfp4kv_cache* cache, int32_t chunk_s
  *   out        device [batch][q_tokens][heads][head_dim], fp32 or bf16 (out_dtype),
  *              contiguous, 16-byte aligned
  *   softmax_scale <= 0 selects 1/sqrt(head_dim)
- *   workspace  device scratch of at least nvfp4kv_workspace_bytes(cache, q_tokens) bytes
- * Chunk slots outside V are never read.  Errors as for nvfp4_kv_quantize; window_chunks < 1,
+ *   workspace  device scratch of at least nvfp4kv_workspace_bytes(cache, q_tokens) bytes (with
+ *              the same device current); contents on entry do not matter
+ * One launch of a persistent kernel (one CTA per SM), followed by a small merge kernel when some
+ * work item's KV tiles were split between CTAs.  Chunk slots outside V are never read.  Errors as for nvfp4_kv_quantize; window_chunks < 1,
  * n_sink_chunks < 0 or q_chunk outside [0, capacity) give NVFP4KV_ERR_INVALID_ARG. */
 int nvfp4_kv_attention(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q_tokens,
                        int64_t q_token_stride, int32_t q_chunk, int32_t n_sink_chunks,
@@ -162,6 +197,23 @@ int nvfp4_kv_attention_slots(const nvfp4kv_cache* cache, const void* q_bf16, int
                              float softmax_scale, void* out, int32_t out_dtype, void* workspace,
                              size_t workspace_bytes, void* cuda_stream);
 
+/* Multi-shot attention sink with the effective key set built inside the library: the paper
+ * page, section 4.2 "Inference with Multi-Shot Attention Sink", and the reading note,
+ * "Multi-shot attention sinks": besides the permanent global sink each shot keeps the chunks
+ * at its start as its own sink, and the query chunk attends to
+ *     K_eff = { c < n_sink_chunks }                                     global sink
+ *           U { shot_start <= c < shot_start + shot_len }               current shot's sink
+ *           U { q_chunk - window_chunks < c <= q_chunk }                sliding window
+ * each slot once.  The shot's sink is history: shot_start >= 0, shot_len >= 0 and
+ * shot_start + shot_len <= q_chunk + 1, else NVFP4KV_ERR_INVALID_ARG (shot_len == 0 gives
+ * nvfp4_kv_attention).  Other arguments, results and errors as for nvfp4_kv_attention; the set
+ * may form at most 4 runs of consecutive slots (it forms at most 3). */
+int nvfp4_kv_attention_multishot(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q_tokens,
+                                 int64_t q_token_stride, int32_t q_chunk, int32_t n_sink_chunks,
+                                 int32_t window_chunks, int32_t shot_start, int32_t shot_len,
+                                 float softmax_scale, void* out, int32_t out_dtype, void* workspace,
+                                 size_t workspace_bytes, void* cuda_stream);
+
 /* Dequantise chunk slots [first_slot, first_slot + n_slots) of K (which == 0) or V
  * (which == 1) into device fp32 out[batch][heads][n_slots*chunk_tokens][head_dim]: the
  * pages' dequantisation step on its own, for tests and diagnostics.  Each value is the
@@ -177,15 +229,24 @@ int nvfp4_kv_dequantize(const nvfp4kv_cache* cache, int32_t which, int32_t first
 int nvfp4kv_debug_encode(const float* x, int64_t n, uint8_t* e2m1_codes, uint8_t* e4m3_codes,
                          void* cuda_stream);
 
-/* The work split nvfp4_kv_attention uses for q_tokens queries on n_sms SMs (n_sms <= 0: the
- * current device's count; any n_sms > 0 needs no GPU).  out[0] = number of CTAs; for 0 <= cta <
- * out[0] also that CTA's work item: out[1] = b * heads + h, out[2] = first query row, out[3] =
- * query tiles of 128 rows (1 or 2, clipped to q_tokens by the kernel).  A host planner chooses how
- * many CTAs take two tiles so that the launch finishes soonest.  A library diagnostic with no
- * counterpart in the pages.  Errors: NVFP4KV_ERR_INVALID_ARG (bad cache, q_tokens <= 0, null out,
- * cta >= out[0]), NVFP4KV_ERR_CUDA (n_sms <= 0 without a device). */
-int nvfp4kv_attention_plan(const nvfp4kv_cache* cache, int32_t q_tokens, int32_t n_sms, int32_t cta,
-                           int32_t* out);
+/* The work split the attention calls use for q_tokens queries over kv_tiles visible KV tiles of
+ * 128 keys on n_sms SMs (n_sms <= 0: the current device's count; any n_sms > 0 needs no GPU).  A
+ * work item is two query tiles of 128 rows of one (batch, head) (the last item of a head holds one
+ * tile when their number is odd) over all kv_tiles KV tiles; the (item, KV tile) units are dealt to
+ * out[0] persistent CTAs as contiguous ranges of equal weighted cost, so a CTA's range is a list of
+ * segments (parts of consecutive items).  A library diagnostic with no counterpart in the pages.
+ *   cta < 0:  out[0] = CTAs, out[1] = kernels per call (2 when some item is split between CTAs and
+ *             the merge kernel runs, else 1)
+ *   cta >= 0: out[0] = CTAs, out[1] = segments of that CTA; for 0 <= seg < out[1] also
+ *             out[2] = batch * heads + head index, out[3] = first query row, out[4] = query tiles
+ *             (1 or 2, clipped to q_tokens by the kernel), [out[5], out[6]) = the KV tiles of the
+ *             item the segment covers, out[7] = its partial-result slot in the workspace, or -1
+ *             when it covers the whole item and writes the output itself
+ * Errors: NVFP4KV_ERR_INVALID_ARG (bad cache, q_tokens or kv_tiles <= 0, null out, cta >= out[0],
+ * seg >= out[1]), NVFP4KV_ERR_UNSUPPORTED (too many units), NVFP4KV_ERR_CUDA (n_sms <= 0 without
+ * a device). */
+int nvfp4kv_attention_plan(const nvfp4kv_cache* cache, int32_t q_tokens, int32_t kv_tiles, int32_t n_sms,
+                           int32_t cta, int32_t seg, int32_t* out);
 
 /* Kernels that nvfp4_kv_quantize (and its static-scratch variant) launch per call for this cache
  * shape on the current device: 1 when every (batch, head, tensor) gets one thread-block cluster

@@ -46,6 +46,9 @@ SIGNATURES = {
     "nvfp4kv_workspace_bytes": (_sz, [_CP, _i32]),
     "nvfp4_kv_quantize": (ctypes.c_int, [_CP, _i32, _vp, _vp, _i64, _vp, _sz, _vp]),
     "nvfp4_kv_quantize_static_scratch": (ctypes.c_int, [_CP, _i32, _vp, _vp, _i64, _vp]),
+    "nvfp4_kv_quantize_layers": (ctypes.c_int, [_CP, _i32, _i32, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i64,
+                                                _vp, _sz, _vp]),
+    "nvfp4kv_quantize_layers_workspace_bytes": (_sz, [_CP, _i32]),
     "nvfp4_kv_attention": (ctypes.c_int, [_CP, _vp, _i32, _i64, _i32, _i32, _i32, ctypes.c_float,
                                           _vp, _i32, _vp, _sz, _vp]),
     "nvfp4_kv_attention_slots": (ctypes.c_int, [_CP, _vp, _i32, _i64, ctypes.POINTER(_i32), _i32,
@@ -53,7 +56,9 @@ SIGNATURES = {
     "nvfp4_kv_dequantize": (ctypes.c_int, [_CP, _i32, _i32, _i32, _vp, _vp]),
     "nvfp4kv_debug_encode": (ctypes.c_int, [_vp, _i64, _vp, _vp, _vp]),
     "nvfp4kv_quantize_launches": (ctypes.c_int, [_CP]),
-    "nvfp4kv_attention_plan": (ctypes.c_int, [_CP, _i32, _i32, _i32, ctypes.POINTER(_i32)]),
+    "nvfp4_kv_attention_multishot": (ctypes.c_int, [_CP, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
+                                                    ctypes.c_float, _vp, _i32, _vp, _sz, _vp]),
+    "nvfp4kv_attention_plan": (ctypes.c_int, [_CP, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_i32)]),
     "nvfp4kv_debug_wait_timeout": (ctypes.c_int, [_CP, _vp]),
     "nvfp4kv_read_status": (ctypes.c_int, [_CP, _vp, ctypes.POINTER(ctypes.c_uint32)]),
     "nvfp4kv_strerror": (ctypes.c_char_p, [ctypes.c_int]),
@@ -121,11 +126,22 @@ def _token_stride(t, name: str, tokens: int, heads: int) -> int:
     return st
 
 
+def workspace_bytes(batch: int, heads: int, chunk_tokens: int, capacity: int, q_tokens: int) -> int:
+    """Scratch bytes the calls on a cache of this shape need on the current device."""
+    d = CacheDesc(batch, heads, HEAD_DIM, chunk_tokens, capacity, 16, 16, 16, 16, 16, 16, 16)
+    n = lib().nvfp4kv_workspace_bytes(ctypes.byref(d), q_tokens)
+    if n == 0:
+        raise NvFp4KvError(ERR_INVALID_ARG, "nvfp4kv_workspace_bytes")
+    return n
+
+
 class KVCache:
     """One layer's NVFP4 KV cache; the arrays are torch CUDA tensors owned by this object."""
 
     def __init__(self, batch: int, heads: int, chunk_tokens: int, capacity: int,
-                 q_tokens_max: int = 0, device=None):
+                 q_tokens_max: int = 0, device=None, workspace=None):
+        """``workspace``: an optional uint8 CUDA tensor used as this cache's scratch instead of one
+        of its own (caches that run on one stream, one call at a time, may share it)."""
         import torch
         self.batch, self.heads, self.chunk_tokens, self.capacity = batch, heads, chunk_tokens, capacity
         dev = torch.device("cuda") if device is None else torch.device(device)
@@ -144,7 +160,8 @@ class KVCache:
                               self.k_scales.data_ptr(), self.v_scales.data_ptr(),
                               self.k_gscale.data_ptr(), self.v_gscale.data_ptr(),
                               self.status.data_ptr())
-        self._ws = None
+        self._ws = workspace
+        self._ws_owned = workspace is None
         self.reserve_workspace(max(q_tokens_max, 1))
 
     def reserve_workspace(self, q_tokens: int) -> None:
@@ -153,6 +170,8 @@ class KVCache:
         if need == 0:
             raise NvFp4KvError(ERR_INVALID_ARG, "nvfp4kv_workspace_bytes")
         if self._ws is None or self._ws.numel() < need:
+            if not self._ws_owned:
+                raise ValueError(f"the shared workspace holds {self._ws.numel()} bytes, {need} are needed")
             self._ws = torch.empty(need, dtype=torch.uint8, device=self.k_codes.device)
 
     @property
@@ -224,14 +243,21 @@ class KVCache:
         return out
 
     def attention_multishot(self, q, q_chunk: int, n_sink: int, window: int, shot_start: int,
-                            shot_len: int, **kw):
-        """Multi-shot attention sink: global sink {c < n_sink}, the current shot's sink
-        {shot_start <= c < shot_start + shot_len} and the window {q_chunk - window < c <= q_chunk}."""
-        if shot_start < 0 or shot_len < 0 or shot_start + shot_len > q_chunk + 1:
-            raise ValueError("the shot sink must lie in [0, q_chunk]")
-        slots = sorted(set(range(min(n_sink, self.capacity))) | set(range(shot_start, shot_start + shot_len)) |
-                       set(range(max(0, q_chunk - window + 1), q_chunk + 1)))
-        return self.attention_slots(q, slots, **kw)
+                            shot_len: int, softmax_scale: float = 0.0, out=None, out_dtype=None,
+                            stream=None):
+        """Multi-shot attention sink: the library attends to the global sink {c < n_sink}, the
+        current shot's sink {shot_start <= c < shot_start + shot_len} and the window
+        {q_chunk - window < c <= q_chunk}, each chunk once."""
+        Lq = q.shape[1]
+        qs = _token_stride(q, "q", Lq, self.heads)
+        out, code = self._out_for(q, out, out_dtype)
+        self.reserve_workspace(Lq)
+        _check(lib().nvfp4_kv_attention_multishot(ctypes.byref(self.desc), q.data_ptr(), Lq, qs, q_chunk,
+                                                  n_sink, window, shot_start, shot_len, float(softmax_scale),
+                                                  out.data_ptr(), code, self._ws.data_ptr(), self._ws.numel(),
+                                                  _stream_handle(stream)),
+               "nvfp4_kv_attention_multishot")
+        return out
 
     def dequantize(self, which: str, first_slot: int = 0, n_slots: int | None = None, stream=None):
         """fp32 [B, H, n_slots*Lc, 128] dequantised K (``which='k'``) or V."""
@@ -250,6 +276,39 @@ class KVCache:
         _check(lib().nvfp4kv_read_status(ctypes.byref(self.desc), _stream_handle(stream), ctypes.byref(v)),
                "nvfp4kv_read_status")
         return v.value
+
+
+def quantize_layers(caches, slot: int, ks, vs, workspace=None, stream=None):
+    """Quantise the new chunk of every layer in one launch: bf16 ``ks[l]``, ``vs[l]``
+    ([B, Lc, H, 128]) into chunk slot ``slot`` of ``caches[l]`` (caches of one shape)."""
+    import torch
+    n = len(caches)
+    if n == 0 or len(ks) != n or len(vs) != n:
+        raise ValueError("one K and one V tensor per cache")
+    c0 = caches[0]
+    strides = {_token_stride(t, "k/v", c0.chunk_tokens, c0.heads) for t in list(ks) + list(vs)}
+    if len(strides) != 1:
+        raise ValueError("every K and V tensor must share one token stride")
+    descs = (CacheDesc * n)(*[c.desc for c in caches])
+    need = lib().nvfp4kv_quantize_layers_workspace_bytes(descs, n)
+    if need == 0:
+        raise NvFp4KvError(ERR_INVALID_ARG, "nvfp4kv_quantize_layers_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=c0.k_codes.device)
+    kp = (_vp * n)(*[t.data_ptr() for t in ks])
+    vp = (_vp * n)(*[t.data_ptr() for t in vs])
+    _check(lib().nvfp4_kv_quantize_layers(descs, n, slot, kp, vp, strides.pop(), workspace.data_ptr(),
+                                          workspace.numel(), _stream_handle(stream)),
+           "nvfp4_kv_quantize_layers")
+    return workspace
+
+
+def attention_plan(cache_desc, q_tokens: int, kv_tiles: int, n_sms: int = 0, cta: int = -1, seg: int = -1):
+    """The attention work split (``nvfp4kv_attention_plan``): a list of 8 ints."""
+    out = (_i32 * 8)()
+    _check(lib().nvfp4kv_attention_plan(ctypes.byref(cache_desc), q_tokens, kv_tiles, n_sms, cta, seg, out),
+           "nvfp4kv_attention_plan")
+    return list(out)
 
 
 def debug_encode(x, stream=None):

@@ -49,7 +49,7 @@ int check_device() {
 
 namespace {
 
-// Checks shared by both attention entry points, then the launch; vis is ascending and distinct.
+// Checks shared by the attention entry points, then the launch; vis is ascending and distinct.
 int attention_checked(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q_tokens,
                       int64_t q_token_stride, const std::vector<int>& vis, float softmax_scale,
                       void* out, int32_t out_dtype, void* workspace, size_t workspace_bytes,
@@ -62,11 +62,16 @@ int attention_checked(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q_
   if (!(softmax_scale == softmax_scale)) return NVFP4KV_ERR_INVALID_ARG;  // NaN
   if (vis.empty()) return NVFP4KV_ERR_INVALID_ARG;
   if (attention_runs(vis) > kAttnMaxRuns) return NVFP4KV_ERR_UNSUPPORTED;
+  int64_t keys = 0;
+  for (size_t i = 0; i < vis.size(); ++i) keys += cache->chunk_tokens;
+  if (!attention_shape_supported(*cache, q_tokens, (keys + 127) / 128 + kAttnMaxRuns))
+    return NVFP4KV_ERR_UNSUPPORTED;
+  const int rc = check_device();
+  if (rc != NVFP4KV_OK) return rc;
+  // the workspace is sized for the current device (one partial-result pair per SM)
   const size_t need = attention_workspace_bytes(*cache, q_tokens);
   if (need > 0 && (!workspace || !aligned16(workspace) || workspace_bytes < need))
     return NVFP4KV_ERR_WORKSPACE;
-  const int rc = check_device();
-  if (rc != NVFP4KV_OK) return rc;
   return launch_attention(*cache, static_cast<const uint16_t*>(q_bf16), q_tokens, q_token_stride, vis,
                           softmax_scale, out, out_dtype, workspace, workspace_bytes,
                           static_cast<cudaStream_t>(cuda_stream));
@@ -114,6 +119,43 @@ int nvfp4_kv_quantize(const nvfp4kv_cache* cache, int32_t chunk_slot, const void
   const cudaError_t e = launch_quantize(*cache, chunk_slot, static_cast<const uint16_t*>(k_bf16),
                                         static_cast<const uint16_t*>(v_bf16), token_stride,
                                         workspace, static_cast<cudaStream_t>(cuda_stream));
+  return e == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
+}
+
+size_t nvfp4kv_quantize_layers_workspace_bytes(const nvfp4kv_cache* caches, int32_t n_layers) {
+  if (!caches || n_layers < 1 || n_layers > 64 || check_cache(&caches[0]) != NVFP4KV_OK) return 0;
+  return quantize_layers_workspace_bytes(n_layers, caches[0].batch, caches[0].heads);
+}
+
+int nvfp4_kv_quantize_layers(const nvfp4kv_cache* caches, int32_t n_layers, int32_t chunk_slot,
+                             const void* const* k_bf16, const void* const* v_bf16, int64_t token_stride,
+                             void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  if (!caches || !k_bf16 || !v_bf16 || n_layers < 1) return NVFP4KV_ERR_INVALID_ARG;
+  int rc = check_cache(&caches[0]);
+  if (rc != NVFP4KV_OK) return rc;
+  const nvfp4kv_cache& c0 = caches[0];
+  if (!quantize_layers_supported(n_layers, c0.batch, c0.heads, c0.chunk_tokens)) return NVFP4KV_ERR_UNSUPPORTED;
+  for (int32_t l = 0; l < n_layers; ++l) {
+    const nvfp4kv_cache& c = caches[l];
+    rc = check_cache(&c);
+    if (rc != NVFP4KV_OK) return rc;
+    if (c.batch != c0.batch || c.heads != c0.heads || c.chunk_tokens != c0.chunk_tokens ||
+        c.capacity_chunks != c0.capacity_chunks)
+      return NVFP4KV_ERR_INVALID_ARG;
+    if (!k_bf16[l] || !v_bf16[l] || !aligned16(k_bf16[l]) || !aligned16(v_bf16[l])) return NVFP4KV_ERR_INVALID_ARG;
+  }
+  if (chunk_slot < 0 || chunk_slot >= c0.capacity_chunks) return NVFP4KV_ERR_INVALID_ARG;
+  if (token_stride < static_cast<int64_t>(c0.heads) * c0.head_dim || token_stride % 8 != 0)
+    return NVFP4KV_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) ||
+      workspace_bytes < quantize_layers_workspace_bytes(n_layers, c0.batch, c0.heads))
+    return NVFP4KV_ERR_WORKSPACE;
+  rc = check_device();
+  if (rc != NVFP4KV_OK) return rc;
+  const cudaError_t e = launch_quantize_layers(caches, n_layers, chunk_slot,
+                                               reinterpret_cast<const uint16_t* const*>(k_bf16),
+                                               reinterpret_cast<const uint16_t* const*>(v_bf16), token_stride,
+                                               workspace, static_cast<cudaStream_t>(cuda_stream));
   return e == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
 }
 
@@ -174,6 +216,30 @@ int nvfp4_kv_attention_slots(const nvfp4kv_cache* cache, const void* q_bf16, int
                            workspace, workspace_bytes, cuda_stream);
 }
 
+int nvfp4_kv_attention_multishot(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q_tokens,
+                                 int64_t q_token_stride, int32_t q_chunk, int32_t n_sink_chunks,
+                                 int32_t window_chunks, int32_t shot_start, int32_t shot_len,
+                                 float softmax_scale, void* out, int32_t out_dtype, void* workspace,
+                                 size_t workspace_bytes, void* cuda_stream) {
+  int rc = check_cache(cache);
+  if (rc != NVFP4KV_OK) return rc;
+  if (q_chunk < 0 || q_chunk >= cache->capacity_chunks || n_sink_chunks < 0 || window_chunks < 1)
+    return NVFP4KV_ERR_INVALID_ARG;
+  // the shot's sink is history of the current shot: it ends at or before the query chunk
+  if (shot_start < 0 || shot_len < 0 || static_cast<int64_t>(shot_start) + shot_len > q_chunk + 1)
+    return NVFP4KV_ERR_INVALID_ARG;
+  // K_eff = global sink U shot sink U window, each slot once, ascending.
+  std::vector<int> vis;
+  for (int ch = 0; ch < cache->capacity_chunks; ++ch) {
+    const bool global_sink = ch < n_sink_chunks;
+    const bool shot_sink = ch >= shot_start && ch < shot_start + shot_len;
+    const bool window = ch > q_chunk - window_chunks && ch <= q_chunk;
+    if (global_sink || shot_sink || window) vis.push_back(ch);
+  }
+  return attention_checked(cache, q_bf16, q_tokens, q_token_stride, vis, softmax_scale, out, out_dtype,
+                           workspace, workspace_bytes, cuda_stream);
+}
+
 int nvfp4_kv_dequantize(const nvfp4kv_cache* cache, int32_t which, int32_t first_slot,
                         int32_t n_slots, float* out, void* cuda_stream) {
   int rc = check_cache(cache);
@@ -209,20 +275,19 @@ int nvfp4kv_debug_wait_timeout(const nvfp4kv_cache* cache, void* cuda_stream) {
              : NVFP4KV_ERR_CUDA;
 }
 
-int nvfp4kv_attention_plan(const nvfp4kv_cache* cache, int32_t q_tokens, int32_t n_sms, int32_t cta,
-                           int32_t* out) {
+int nvfp4kv_attention_plan(const nvfp4kv_cache* cache, int32_t q_tokens, int32_t kv_tiles, int32_t n_sms,
+                           int32_t cta, int32_t seg, int32_t* out) {
   int rc = check_cache(cache);
   if (rc != NVFP4KV_OK) return rc;
-  if (q_tokens <= 0 || !out) return NVFP4KV_ERR_INVALID_ARG;
+  if (q_tokens <= 0 || q_tokens > (1 << 24) || kv_tiles <= 0 || !out) return NVFP4KV_ERR_INVALID_ARG;
+  if (!attention_shape_supported(*cache, q_tokens, kv_tiles)) return NVFP4KV_ERR_UNSUPPORTED;
   if (n_sms <= 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return NVFP4KV_ERR_CUDA;
+    n_sms = current_sm_count();
+    if (n_sms <= 0) return NVFP4KV_ERR_CUDA;
   }
-  int o[4];
-  rc = attention_plan(*cache, q_tokens, n_sms, cta, o);
-  for (int i = 0; i < 4; ++i) out[i] = o[i];
+  int o[8];
+  rc = attention_plan(*cache, q_tokens, kv_tiles, n_sms, cta, seg, o);
+  for (int i = 0; i < 8; ++i) out[i] = o[i];
   return rc;
 }
 

@@ -7,25 +7,33 @@
 // 2.1: a chunk sees its own tokens.  Reading note (yingwang.github.io), "The NVFP4
 // quantization format": x_hat = E2M1 * E4M3 * FP32 scale.
 //
-// One CTA owns one or two query tiles of 128 rows of one (batch, head) and walks the visible
-// KV tiles (128 keys each; tiles lie inside runs of consecutive visible chunks, so chunks
-// outside the mask are never read).  A host planner chooses how many CTAs take two tiles.
+// Work: every (batch, head) has ceil(Lq / 128) query tiles, grouped into work items of two tiles
+// (the last item of a head holds one tile when the count is odd); an item walks all visible KV
+// tiles (128 keys each; tiles lie inside runs of consecutive visible chunks, so chunks outside
+// the mask are never read).  The grid is persistent: one CTA per SM, and the (item, KV tile)
+// units are dealt out as equal-cost contiguous ranges (stream-K), so a CTA may finish one item,
+// run a whole item, and start another.  A range that covers only part of an item's KV tiles
+// leaves a partial result (unnormalised O, running max, running sum) in the workspace, and
+// combine_kernel merges the parts of every split item.
+//
 // 512 threads, four warpgroups; warp roles:
-//   softmax warps 0-3, 4-7    query tile 0 / 1: one query row per thread, online softmax over
-//                             TMEM rows, epilogue (176 registers each, setmaxnreg)
-//   producer warp 8           TMA: Q tiles (tensor map, 128B swizzle) and packed K/V tiles
-//                             + E4M3 scales (1-D bulk copies) into a ring of smem slots
-//   MMA warp 9                TMEM allocation; tcgen05.mma S = Q K^T (both operands in
-//                             smem), O += P V (P from TMEM, V from smem), eight MMAs per asm
-//                             block from one elected lane
+//   softmax warps 0-3, 4-7    query tile 0 / 1 of the item: one query row per thread, online
+//                             softmax over TMEM rows, epilogue; each warpgroup loads its own Q
+//                             tile (TMA, 128B swizzle) and converts it to fp16 in place
+//   producer warp 8           1-D bulk copies of each KV tile's packed codes + E4M3 scales into
+//                             a ring of shared-memory slots
+//   MMA warp 9                TMEM allocation; tcgen05.mma S = Q K^T (both operands in smem),
+//                             O += P V (P from TMEM, V from smem), one elected lane
 //   dequant warps 10-15       E2M1 * E4M3 products, exact in fp16, written straight into the
 //                             128B-swizzled UMMA operand layout: K (the B operand of Q K^T,
 //                             K-major) and V (the B operand of P V, MN-major)
-// With two tiles the softmax warpgroups alternate with the tensor core: PV(0, j), QK(0, j+1),
-// PV(1, j), QK(1, j+1).  The FP32 scales stay out of the MMAs: g_K(chunk) multiplies S per
-// column, and g_V(chunk) / max g_V multiplies P per column before P is rounded to fp16 (fp16
-// P and V keep the P V product 8x finer than bf16).  Rows are rescaled lazily: the running
-// max only moves when it grows by more than 2^8.
+// S is computed in sub-tiles of 64 keys, double-buffered in TMEM per query tile (4 x 64 columns
+// of S, 2 x 128 columns of O): while the softmax warps work on sub-tile h, the tensor core
+// already holds S of sub-tile h + 1, so the softmax never waits on the MMA chain.  The FP32
+// scales stay out of the MMAs: g_K(chunk) multiplies S per column, and g_V(chunk) / max g_V
+// multiplies P per column before P is rounded to fp16 (fp16 P and V keep the P V product 8x
+// finer than bf16).  Rows are rescaled lazily: the running max only moves when it grows by more
+// than 2^8.
 //
 // Every mbarrier wait is bounded (%globaltimer); on a time-out the kernel ORs
 // NVFP4KV_ERR_DEVICE_TIMEOUT into the status word, lets in-flight copies and MMAs finish,
@@ -35,9 +43,6 @@
 
 #include <algorithm>
 #include <cmath>
-#include <map>
-#include <mutex>
-#include <tuple>
 #include <vector>
 
 #include "internal.h"
@@ -48,18 +53,23 @@ namespace {
 
 constexpr int BM = 128;  // query rows per tile (TMEM lanes)
 constexpr int BN = 128;  // keys per KV tile
+constexpr int SUB = 64;  // keys per S sub-tile
 constexpr int D = kHeadDim;
+constexpr int QT = 2;    // query tiles per work item
 constexpr int NST = 2;   // stages of dequantised K / V tiles
 constexpr int NPK = 3;   // slots of packed data (K and V tiles alternate)
 constexpr int NCT = 4;   // slots of per-tile column tables
-constexpr int kMaxTabChunks = 256;  // chunk scales staged in shared memory up to this many slots
 constexpr int PK_CODES = BN * kCodeBytes;               // 8192
 constexpr int PK_BYTES = PK_CODES + BN * kScaleBytes;   // 9216
 constexpr int TILE16 = BN * D * 2;                      // one 128 x 128 16-bit operand tile
 constexpr int HALF16 = TILE16 / 2;                      // 128 rows x 64 elements (128 B rows)
 constexpr int MAX_RUNS = kAttnMaxRuns;
+constexpr int kMaxCtas = 1024;
+// Relative cost of one KV tile of a two-tile item and of a one-tile item (the planner's weights).
+constexpr int kWPair = 5, kWSingle = 3;
+// Floats of one partial-result slot: O[QT][BM][D], m[QT][BM], l[QT][BM], the reference g_V.
+constexpr int kSlotFloats = QT * BM * D + 2 * QT * BM + 4;
 
-template <int QT>
 struct Cfg {
   static constexpr int kSoftmaxWarps = 4 * QT;
   static constexpr int kProducerWarp = kSoftmaxWarps;
@@ -69,38 +79,94 @@ struct Cfg {
   static constexpr int kDequantThreads = 32 * kDequantWarps;
   static_assert(kDequantThreads % 64 == 0, "dequant_tile deals blocks to a multiple of 64 threads");
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 2 + kDequantWarps);  // whole warpgroups
-  static constexpr uint32_t kTmemCols = QT == 1 ? 256 : 512;
+  static_assert(kThreads == 512, "register split assumes four warpgroups");
+  // TMEM columns: S sub-tile buffers S[q][b] at (2q + b) * SUB, O[q] at kTmemO + q * D.
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kTmemO = 2 * QT * SUB;
+  static_assert(kTmemO + QT * D <= kTmemCols, "TMEM budget");
   // shared memory map (bytes from a 1024-aligned base)
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + QT * TILE16;
   static constexpr int oV = oK + NST * TILE16;
   static constexpr int oPK = oV + NST * TILE16;
-  // Per-tile column tables colK[BN], colV[BN] (fp32) and int4 {n_valid, uniform}, in NCT slots:
-  // the K stage of tile j is refilled once the QKs of tile j - NST are done, while the softmax
-  // warps may still read the tables of tiles j - NST and j - NST + 1.
+  // Per-tile column tables (fp32, BN each): K[j] = g_K(chunk) * scale * log2(e), L[j] = log2(cv),
+  // I[j] = 1 / cv with cv = g_V(chunk) / max g_V (1 for an all-zero V chunk, whose V^ rows are 0);
+  // masked columns K = 0, L = -inf, I = 0.  Plus int4 {n_valid, uniform}.  NCT slots.
+  static constexpr int kColTab = 3 * BN * 4;
   static constexpr int oCol = oPK + NPK * PK_BYTES;
-  static constexpr int oInfo = oCol + NCT * 2 * BN * 4;
-  static constexpr int oRed = oInfo + NCT * 16;          // per Q tile: 4 warp maxima
-  static constexpr int oTab = oRed + QT * 16;            // per chunk slot: {g_K * scale, g_V / max g_V}
-  static constexpr int oBar = oTab + kMaxTabChunks * 8;
+  static constexpr int oInfo = oCol + NCT * kColTab;
+  static constexpr int oBar = oInfo + NCT * 16;
   // barrier indices
-  static constexpr int bQFull = 0;
-  static constexpr int bQReady = 1;
-  static constexpr int bPkFull = 2;
-  static constexpr int bPkEmpty = bPkFull + NPK;
-  static constexpr int bKFull = bPkEmpty + NPK;
-  static constexpr int bVFull = bKFull + NST;
-  static constexpr int bKEmpty = bVFull + NST;  // K stage read by every QK of its tile
-  static constexpr int bVEmpty = bKEmpty + NST;  // V stage read by every PV of its tile
-  static constexpr int bSFull = bVEmpty + NST;
-  static constexpr int bPFull = bSFull + QT;
-  static constexpr int bODone = bPFull + QT;
-  static constexpr int bDrain = bODone + QT;
+  static constexpr int bQFull = 0;                 // [QT] Q tile landed (TMA)
+  static constexpr int bQReady = bQFull + QT;      // [QT] Q tile converted to fp16
+  static constexpr int bPkFull = bQReady + QT;     // [NPK]
+  static constexpr int bPkEmpty = bPkFull + NPK;   // [NPK]
+  static constexpr int bKFull = bPkEmpty + NPK;    // [NST]
+  static constexpr int bVFull = bKFull + NST;      // [NST]
+  static constexpr int bKEmpty = bVFull + NST;     // [NST] K stage read by every QK of its tile
+  static constexpr int bVEmpty = bKEmpty + NST;    // [NST] V stage read by every PV of its tile
+  static constexpr int bTabFull = bVEmpty + NST;   // [NCT] column tables of a tile written
+  static constexpr int bSFull = bTabFull + NCT;    // [QT][2] S sub-tile computed
+  static constexpr int bPFull = bSFull + 2 * QT;   // [QT][2] P sub-tile stored
+  static constexpr int bODone = bPFull + 2 * QT;   // [QT][2] PV of a sub-tile complete
+  static constexpr int bDrain = bODone + 2 * QT;
   static constexpr int kNumBars = bDrain + 1;
   static constexpr int oMisc = oBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag
   static constexpr int kSmemBytes = oMisc + 16 + 1024;  // + slack for 1024-B alignment
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
+
+// The stream-K work split: units are (work item, KV tile) pairs, numbered item-major; a unit of
+// a two-tile item costs wP, of a one-tile item wS.  CTA c takes the units whose weighted start
+// lies in [c W / G, (c + 1) W / G).
+struct Plan {
+  int64_t units;  // bh * ipb * NT
+  int64_t Wh;     // weighted cost of one (batch, head)
+  int64_t W;      // bh * Wh
+  int bh;         // batch * heads
+  int n_qt;       // query tiles per (batch, head)
+  int ipb;        // work items per (batch, head): ceil(n_qt / 2)
+  int npairs;     // two-tile items per (batch, head): n_qt / 2
+  int NT;         // KV tiles per item
+  int wP, wS;
+  int G;          // CTAs
+};
+
+// First unit of CTA c (c = G gives the end of the last range).
+__host__ __device__ inline int64_t plan_cut(const Plan& p, int c) {
+  if (c <= 0) return 0;
+  if (c >= p.G) return p.units;
+  const int64_t X = (p.W / p.G) * c + ((p.W % p.G) * c) / p.G;  // floor(W c / G)
+  const int64_t h = X / p.Wh, r = X - h * p.Wh;
+  const int64_t pw = static_cast<int64_t>(p.NT) * p.wP * p.npairs;
+  int64_t u;
+  if (r <= pw) u = (r + p.wP - 1) / p.wP;
+  else u = static_cast<int64_t>(p.NT) * p.npairs + (r - pw + p.wS - 1) / p.wS;
+  return h * p.ipb * static_cast<int64_t>(p.NT) + u;
+}
+
+// One segment of a CTA's range: the part of one work item between units u and uend.  Unit
+// numbers stay below 2^31 (the launch checks it), so segments use 32-bit arithmetic.
+struct Seg {
+  int item;
+  int t0, t1;  // KV tiles [t0, t1) of the item
+  int bhi, m0, nq;
+};
+
+__host__ __device__ inline Seg plan_seg(const Plan& p, int u, int uend) {
+  Seg s;
+  s.item = u / p.NT;
+  const int ib = s.item * p.NT;
+  s.t0 = u - ib;
+  s.t1 = (uend < ib + p.NT ? uend : ib + p.NT) - ib;
+  s.bhi = s.item / p.ipb;
+  const int k = s.item - s.bhi * p.ipb;
+  s.m0 = 2 * k * BM;
+  s.nq = (2 * k + 1 < p.n_qt) ? 2 : 1;
+  return s;
+}
+
+__host__ __device__ inline int seg_end(const Plan& p, const Seg& s) { return s.item * p.NT + s.t1; }
 
 struct AttnParams {
   const uint8_t* k_codes;
@@ -110,6 +176,7 @@ struct AttnParams {
   const float* k_g;
   const float* v_g;
   void* out;
+  float* part;  // partial-result slots: [G][2][kSlotFloats]
   uint32_t* status;
   int64_t T;  // cached tokens per (b, h)
   int B, H, Lq, Lc, C;
@@ -120,10 +187,7 @@ struct AttnParams {
   int run_tile0[MAX_RUNS + 1];
   int n_tiles;
   float scale_log2;  // softmax scale * log2(e)
-  // Work list: every (b, h) has n_qt query tiles of 128 rows; the first pp + 1 (for (b, h) <
-  // pr) or pp of its tile pairs go to two-tile CTAs, the rest of its tiles to one-tile CTAs.
-  // CTAs [0, n_pair_ctas) take pairs, the others single tiles.
-  int n_qt, pp, pr, n_pair_ctas;
+  Plan pl;
 };
 
 // ------------------------------------------------------------------ waits
@@ -214,7 +278,7 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
 template <int NT, bool kFull>
 __device__ __forceinline__ void dequant_tile(const uint8_t* pk, uint8_t* dst, int n, int dt) {
   static_assert(NT % 64 == 0, "keys per pass must be a multiple of 8");
-  constexpr int KS = NT / 8;               // keys per pass: 24 for 192 threads, 40 for 320
+  constexpr int KS = NT / 8;               // keys per pass: 24 for 192 threads
   constexpr int kIt = (BN + KS - 1) / KS;  // passes; the last one may cover only part of the keys
   const int blk = dt & 7, kq = dt >> 3;
   const bool swap = blk >= 4;
@@ -224,7 +288,7 @@ __device__ __forceinline__ void dequant_tile(const uint8_t* pk, uint8_t* dst, in
   uint8_t* const row = dst + (blk >> 2) * HALF16 + kq * 128;
   uint8_t* const dA = row + (((c0 + (swap ? 1 : 0)) ^ (kq & 7)) << 4);  // first store
   uint8_t* const dB = row + (((c0 + (swap ? 0 : 1)) ^ (kq & 7)) << 4);
-  const bool tail = kq + KS * (kIt - 1) < BN;  // this thread has a sixth key
+  const bool tail = kq + KS * (kIt - 1) < BN;  // this thread has a key in the last pass
   uint2 w[kIt];
   uint32_t sb[kIt];
 #pragma unroll
@@ -255,62 +319,17 @@ __device__ __forceinline__ void dequant_tile(const uint8_t* pk, uint8_t* dst, in
   }
 }
 
-// Work item of CTA c: every (b, h) has n_qt query tiles; (b, h) < pr gives its first pp + 1 tile
-// pairs to two-tile CTAs, the others their first pp; CTAs [0, n_pair_ctas) take those pairs in
-// (b, h) order, the rest take the remaining tiles one by one, also in (b, h) order.  Shared by the
-// kernel and the host diagnostic that checks the split.
-struct WorkItem {
-  int bhi, m0, nq;
-};
-
-__host__ __device__ inline WorkItem work_item(int c, int n_qt, int pp, int pr, int n_pair_ctas) {
-  WorkItem w;
-  if (c < n_pair_ctas) {
-    const int big = pr * (pp + 1);
-    int idx;
-    if (c < big || pp == 0) {
-      w.bhi = c / (pp + 1);
-      idx = c % (pp + 1);
-    } else {
-      w.bhi = pr + (c - big) / pp;
-      idx = (c - big) % pp;
-    }
-    w.m0 = idx * 2 * BM;
-    w.nq = 2;
-  } else {
-    const int c2 = c - n_pair_ctas;
-    const int s_big = n_qt - 2 * (pp + 1), s_small = n_qt - 2 * pp;
-    const int big = s_big > 0 ? pr * s_big : 0;
-    int idx, pairs;
-    if (c2 < big || s_small <= 0) {
-      w.bhi = s_big > 0 ? c2 / s_big : 0;
-      idx = s_big > 0 ? c2 % s_big : 0;
-      pairs = pp + 1;
-    } else {
-      w.bhi = pr + (c2 - big) / s_small;
-      idx = (c2 - big) % s_small;
-      pairs = pp;
-    }
-    w.m0 = (2 * pairs + idx) * BM;
-    w.nq = 1;
-  }
-  return w;
-}
-
-template <int QT>
-__global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
+__global__ void __launch_bounds__(Cfg::kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ AttnParams p) {
-  using C = Cfg<QT>;
+  using C = Cfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // This CTA's work item: (b, h), first query row m0 and nq query tiles.
-  const WorkItem wi = work_item(blockIdx.x, p.n_qt, p.pp, p.pr, p.n_pair_ctas);
-  const int bhi = wi.bhi, m0 = wi.m0, nq = wi.nq;
-  const int h = bhi % p.H, b = bhi / p.H;
-  const int64_t bh = static_cast<int64_t>(b) * p.H + h;
+  const int cta = blockIdx.x;
+  // This CTA's range of (item, KV tile) units; every role walks the same segments.
+  const int ubeg = static_cast<int>(plan_cut(p.pl, cta)), uend = static_cast<int>(plan_cut(p.pl, cta + 1));
   const int n_dq_warps = C::kDequantWarps;
 
   const uint32_t sbase = ptx::smem_u32(smem);
@@ -319,8 +338,15 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
   volatile uint32_t* abort_flag = misc + 1;
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(bar(C::bQFull), 1);
-    ptx::mbar_init(bar(C::bQReady), 4 * nq);
+    for (int q = 0; q < QT; ++q) {
+      ptx::mbar_init(bar(C::bQFull + q), 1);
+      ptx::mbar_init(bar(C::bQReady + q), 4);
+      for (int b = 0; b < 2; ++b) {
+        ptx::mbar_init(bar(C::bSFull + 2 * q + b), 1);
+        ptx::mbar_init(bar(C::bPFull + 2 * q + b), 4);
+        ptx::mbar_init(bar(C::bODone + 2 * q + b), 1);
+      }
+    }
     for (int i = 0; i < NPK; ++i) {
       ptx::mbar_init(bar(C::bPkFull + i), 1);
       ptx::mbar_init(bar(C::bPkEmpty + i), n_dq_warps);
@@ -331,11 +357,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       ptx::mbar_init(bar(C::bKEmpty + i), 1);
       ptx::mbar_init(bar(C::bVEmpty + i), 1);
     }
-    for (int q = 0; q < QT; ++q) {
-      ptx::mbar_init(bar(C::bSFull + q), 1);
-      ptx::mbar_init(bar(C::bPFull + q), 4);
-      ptx::mbar_init(bar(C::bODone + q), 1);
-    }
+    for (int i = 0; i < NCT; ++i) ptx::mbar_init(bar(C::bTabFull + i), n_dq_warps);
     ptx::mbar_init(bar(C::bDrain), 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -349,104 +371,79 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = misc[0];
-  // Registers move from the producer/MMA/dequant warpgroups (80 each) to the two softmax
-  // warpgroups (176 each), which hold a whole 128-column S row: 2*128*176 + 2*128*80 = 65536,
-  // exactly what the 512-thread block was launched with.  Each role branch starts with its
-  // warpgroup's budget change.
-  static_assert(QT == 1 || C::kThreads == 512, "register split assumes four warpgroups");
-
-  // Dequantiser role: thread dt of the nthreads threads of the dequant warps.
-  auto dequant_role = [&](int dt) {
-    const int nthreads = 32 * n_dq_warps;
-    const float inv_gv = 1.0f / max_visible_gv(p, bh);
-    // The per-chunk FP32 scales of this (b, h), staged once, so the per-tile column tables are
-    // built from shared memory.
-    const float2* gtab = reinterpret_cast<const float2*>(smem + C::oTab);
-    const bool use_tab = p.C <= kMaxTabChunks;
-    if (use_tab)
-      for (int c = dt; c < p.C; c += nthreads)
-        reinterpret_cast<float2*>(smem + C::oTab)[c] =
-            make_float2(p.k_g[bh * p.C + c] * p.scale_log2, p.v_g[bh * p.C + c] * inv_gv);
-    ptx::named_bar(3, nthreads);
-    bool ok = true;
-    for (int j = 0; j < p.n_tiles && ok; ++j) {
-      const int st = j % NST;
-      int key0, n;
-      tile_keys(p, j, key0, n);
-      for (int t = 0; t < 2 && ok; ++t) {
-        // the stage's previous tile (j - NST) is done with it: K after its QKs, V after its PVs
-        if (j >= NST) ok = waitw(bar((t == 0 ? C::bKEmpty : C::bVEmpty) + st), ((j / NST) - 1) & 1, abort_flag, p.status);
-        if (!ok) break;
-        const int pk = 2 * j + t;
-        const int slot = pk % NPK;
-        ok = waitw(bar(C::bPkFull + slot), (pk / NPK) & 1, abort_flag, p.status);
-        if (!ok) break;
-        const uint8_t* src = smem + C::oPK + slot * PK_BYTES;
-        uint8_t* dst = smem + (t == 0 ? C::oK : C::oV) + st * TILE16;
-        if (n == BN) dequant_tile<C::kDequantThreads, true>(src, dst, n, dt);
-        else dequant_tile<C::kDequantThreads, false>(src, dst, n, dt);
-        if (t == 0 && dt < BN) {  // per-column tables: one thread per key of the tile
-          float* colK = reinterpret_cast<float*>(smem + C::oCol + (j % NCT) * 2 * BN * 4);
-          const bool valid = dt < n;
-          const int c = valid ? (key0 + dt) / p.Lc : 0;
-          const float2 g = !valid ? make_float2(0.0f, 0.0f)
-                           : use_tab ? gtab[c]
-                                     : make_float2(p.k_g[bh * p.C + c] * p.scale_log2, p.v_g[bh * p.C + c] * inv_gv);
-          colK[dt] = g.x;
-          colK[BN + dt] = g.y;
-          if (dt == 0) {
-            const int uniform = (n == BN) && (key0 / p.Lc == (key0 + BN - 1) / p.Lc);
-            *reinterpret_cast<int4*>(smem + C::oInfo + 16 * (j % NCT)) = make_int4(n, uniform, 0, 0);
-          }
-        }
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          ptx::mbar_arrive(bar(C::bPkEmpty + slot));
-          ptx::mbar_arrive(bar(t == 0 ? C::bKFull + st : C::bVFull + st));
-        }
-      }
-    }
-  };
+  // Registers move from the producer/MMA/dequant warpgroups (88 each) to the two softmax
+  // warpgroups (168 each): 2*128*168 + 2*128*88 = 65536, exactly what the 512-thread block was
+  // launched with.  Each role branch starts with its warpgroup's budget change.
 
   if (warp < C::kSoftmaxWarps) {
     // ============================================================ softmax + epilogue
-    if constexpr (QT == 2) ptx::setmaxnreg_inc<176>();
+    ptx::setmaxnreg_inc<168>();
     const int qt = warp >> 2;
-    if (qt < nq) {
-    const int row = (warp & 3) * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_off + qt * BN;
-    const uint32_t tO = tmem + lane_off + QT * BN + qt * D;
-    const float gv_ref = max_visible_gv(p, bh);
-    bool ok = waitw(bar(C::bQFull), 0, abort_flag, p.status);
-    float pre_scale = 1.0f;
-
-    // ---- Q tile: bf16 -> fp16 in place, exact, after a power-of-two prescale 2^-e that keeps
-    // the tile's largest |q| below 2^15; S is scaled back by 2^e with the logit factor.
-    float q_unscale = 1.0f;
-    uint8_t* qrow = smem + C::oQ + qt * TILE16 + row * 128;
-    {
-      uint32_t mb = 0;
-      if (ok) {
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS0 = tmem + lane_off + (2 * qt) * SUB;
+    const uint32_t tO = tmem + lane_off + C::kTmemO + qt * D;
+    const bool issuer = wq == 0 && lane == 0;
+    uint8_t* const qbase = smem + C::oQ + qt * TILE16;
+    // The Q tile of the next segment this warpgroup takes part in, loaded by one thread.
+    auto issue_q = [&](int from) {
+      for (int u = from; u < uend;) {
+        const Seg s = plan_seg(p.pl, u, uend);
+        if (qt < s.nq) {
+          if (issuer) {
+            const int hh = s.bhi % p.H, bb = s.bhi / p.H;
+            ptx::mbar_arrive_expect_tx(bar(C::bQFull + qt), TILE16);
+            for (int half = 0; half < 2; ++half)
+              ptx::tma_load_4d(sbase + C::oQ + qt * TILE16 + half * HALF16, &tmap_q, half * 64, hh,
+                               s.m0 + qt * BM, bb, bar(C::bQFull + qt));
+          }
+          return true;
+        }
+        u = seg_end(p.pl, s);
+      }
+      return false;
+    };
+    if (issuer) ptx::prefetch_tmap(&tmap_q);
+    bool q_pending = issue_q(ubeg);
+    bool ok = true;
+    int sq = 0;        // segments this warpgroup took part in
+    int g = 0;         // S sub-tiles this warpgroup processed (parity of its S/P/O barriers)
+    int jjb = 0;       // KV tiles of the CTA before the current segment
+    for (int u = ubeg; u < uend && ok;) {
+      const Seg s = plan_seg(p.pl, u, uend);
+      const int unext = seg_end(p.pl, s);
+      const int ntl = s.t1 - s.t0;
+      if (qt >= s.nq) {
+        jjb += ntl;
+        u = unext;
+        continue;
+      }
+      const int h = s.bhi % p.H, b = s.bhi / p.H;
+      const int64_t bh = static_cast<int64_t>(b) * p.H + h;
+      ok = waitw(bar(C::bQFull + qt), sq & 1, abort_flag, p.status);
+      if (!ok) break;
+      q_pending = false;
+      // ---- Q row: bf16 -> fp16 in place after a power-of-two prescale 2^-e that keeps the row's
+      // largest |q| below 2^15; row i of S depends on row i of Q only, so each thread scales its
+      // own row and scales its S row back by 2^e with the logit factor.  The conversion is exact
+      // for elements >= 2^(e-14) (fp16's normal range); smaller ones round to fp16's subnormal
+      // spacing 2^(e-24).  No thread waits for another here.
+      float q_unscale = 1.0f, pre_scale = 1.0f;
+      uint8_t* qrow = qbase + row * 128;
+      {
+        uint32_t mb = 0;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const uint4 v = *reinterpret_cast<const uint4*>(qrow + (i >> 3) * HALF16 + (((i + lane) & 7) << 4));
           mb = __vmaxu2(mb, __vmaxu2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w)));
         }
+        mb = max(mb & 0xFFFFu, mb >> 16);
+        const int ex = static_cast<int>((mb >> 7) & 0xFF) - 127;  // floor(log2 max|q|)
+        const int e = ex > 14 ? ex - 14 : 0;
+        q_unscale = __int_as_float((127 + e) << 23);  // 2^e
+        pre_scale = __int_as_float((127 - e) << 23);  // 2^-e
       }
-      mb = max(mb & 0xFFFFu, mb >> 16);
-      mb = __reduce_max_sync(0xFFFFFFFFu, mb);
-      uint32_t* red = reinterpret_cast<uint32_t*>(smem + C::oRed + qt * 16);
-      if (lane == 0) red[warp & 3] = mb;
-      ptx::named_bar(1 + qt, 128);  // reached by all four warps of the tile, on every path
-      mb = max(max(red[0], red[1]), max(red[2], red[3]));
-      const int ex = static_cast<int>((mb >> 7) & 0xFF) - 127;  // floor(log2 max|q|)
-      const int e = ex > 14 ? ex - 14 : 0;
-      q_unscale = __int_as_float((127 + e) << 23);  // 2^e
-      pre_scale = __int_as_float((127 - e) << 23);  // 2^-e
-    }
-    if (ok) {
 #pragma unroll 4
       for (int i = 0; i < 16; ++i) {
         uint4* ptr = reinterpret_cast<uint4*>(qrow + (i >> 3) * HALF16 + (((i + lane) & 7) << 4));
@@ -461,148 +458,168 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       }
       ptx::fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(C::bQReady));
-    }
+      if (lane == 0) ptx::mbar_arrive(bar(C::bQReady + qt));
 
-    float m_run = -INFINITY, l_run = 0.0f;
-    for (int j = 0; j < p.n_tiles && ok; ++j) {
-      const int st = j % NST;
-      ok = waitw(bar(C::bSFull + qt), j & 1, abort_flag, p.status) &&
-           waitw(bar(C::bKFull + st), (j / NST) & 1, abort_flag, p.status);
+      const float gv_ref = max_visible_gv(p, bh);
+      float m_run = -INFINITY, l_run = 0.0f;
+      const int nh = 2 * ntl;
+      for (int hs = 0; hs < nh && ok; ++hs, ++g) {
+        const int jj = jjb + (hs >> 1);
+        const int bf = g & 1, half = hs & 1;
+        const uint32_t tS = tS0 + bf * SUB;
+        ok = waitw(bar(C::bSFull + 2 * qt + bf), (g >> 1) & 1, abort_flag, p.status);
+        if (ok && half == 0) ok = waitw(bar(C::bTabFull + jj % NCT), (jj / NCT) & 1, abort_flag, p.status);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const int ct = static_cast<int>(jj % NCT);
+        const int4 info = *reinterpret_cast<const int4*>(smem + C::oInfo + 16 * ct);
+        const float* colK = reinterpret_cast<const float*>(smem + C::oCol + ct * C::kColTab) + half * SUB;
+        const float* colL = colK + BN;
+        const float* colI = colK + 2 * BN;
+        // A tile inside one chunk with every key valid takes the uniform path (one logit factor,
+        // one cv); any other tile works per column with the same arithmetic.
+        const bool uni = info.y != 0;
+
+        uint32_t sr[2][32];
+        ptx::tmem_ld32(tS, sr[0]);
+        ptx::tmem_ld32(tS + 32, sr[1]);
+        ptx::tc_wait_ld_regs(sr[0]);
+        ptx::reg_fence32(sr[1]);
+
+        // Row maximum of x = S * g_K(chunk) * scale * log2(e) + log2(cv) (masked keys -inf); the
+        // reference m only has to bound the exponents of P~ = 2^(x - m), which include cv.
+        float mx;
+        float ck = 0.0f, lc = 0.0f;
+        if (uni) {
+          ck = colK[0] * q_unscale;
+          lc = colL[0];
+          float m8[8];  // eight independent max chains
+#pragma unroll
+          for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const int k = 4 * c + ((i >> 2) & 1) * 2;
+              m8[k] = ptx::fmax3(m8[k], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
+              m8[k + 1] = ptx::fmax3(m8[k + 1], __uint_as_float(sr[c][i + 2]), __uint_as_float(sr[c][i + 3]));
+            }
+          mx = fmaf(fmaxf(ptx::fmax3(m8[0], m8[1], m8[2]), ptx::fmax3(m8[3], m8[4], ptx::fmax3(m8[5], m8[6], m8[7]))),
+                    ck, lc);
+        } else {
+          // x in place of S: x = S * K[j] * 2^e + L[j]
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              asm volatile("" ::: "memory");  // keep the table loads next to their use (registers)
+              const float4 kk = *reinterpret_cast<const float4*>(colK + 32 * c + i);
+              const float4 ll = *reinterpret_cast<const float4*>(colL + 32 * c + i);
+              const float x0 = fmaf(__uint_as_float(sr[c][i]), kk.x * q_unscale, ll.x);
+              const float x1 = fmaf(__uint_as_float(sr[c][i + 1]), kk.y * q_unscale, ll.y);
+              const float x2 = fmaf(__uint_as_float(sr[c][i + 2]), kk.z * q_unscale, ll.z);
+              const float x3 = fmaf(__uint_as_float(sr[c][i + 3]), kk.w * q_unscale, ll.w);
+              sr[c][i] = __float_as_uint(x0);
+              sr[c][i + 1] = __float_as_uint(x1);
+              sr[c][i + 2] = __float_as_uint(x2);
+              sr[c][i + 3] = __float_as_uint(x3);
+              m4[(i >> 2) & 3] = fmaxf(m4[(i >> 2) & 3], ptx::fmax3(x0, x1, fmaxf(x2, x3)));
+            }
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        }
+        // Lazy rescale: the reference m only moves (to a whole number, so the rescale is an exact
+        // power of two) when the row maximum exceeds it by more than 2^8.  The O rescale uses
+        // warp-collective TMEM accesses, so it runs for the whole warp when any row moved
+        // (alpha = 1 for the rows that did not).
+        const bool grow = mx > m_run + 8.0f;
+        if (__any_sync(0xFFFFFFFFu, grow)) {
+          const float m_new = grow ? ceilf(mx) : m_run;
+          const float alpha = grow ? ptx::ex2(m_run - m_new) : 1.0f;  // 0 while m is -inf
+          l_run *= alpha;
+          m_run = m_new;
+          if (hs > 0) {  // O holds sub-tiles < hs of this segment once PV(g - 1) is complete
+            ok = waitw(bar(C::bODone + 2 * qt + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, p.status);
+            if (!ok) break;
+            ptx::tc_fence_after();
+#pragma unroll 1
+            for (int oc = 0; oc < 8; ++oc) {  // 16 columns at a time: the S row stays in registers
+              uint32_t o[16];
+              ptx::tmem_ld16_wait(tO + 16 * oc, o);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              ptx::tmem_st16p(tO + 16 * oc, o);
+            }
+          }
+        }
+
+        // P~ = 2^(x - m) (x includes log2(cv)), rounded to fp16 pairs and stored over the
+        // sub-tile's first 32 S columns.  The row sum adds the same rounded values times 1 / cv,
+        // so the rounding largely cancels in O / l.
+        if (uni) {
+          // x - m = S * ck + (log2(cv) - m) in packed pairs; eight independent row-sum chains.
+          const float mneg = lc - m_run;
+          float l8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) l8[k] = 0.0f;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float x0, x1;
+              ptx::ffma2(x0, x1, __uint_as_float(sr[c][2 * i]), __uint_as_float(sr[c][2 * i + 1]), ck, mneg);
+              pk[i] = ptx::f32x2_to_f16x2(ptx::ex2(x0), ptx::ex2(x1));
+              l8[i & 7] = ptx::add_f16x2_f32(l8[i & 7], pk[i]);
+            }
+            ptx::tmem_st16p(tS + 16 * c, pk);
+          }
+          l_run = fmaf((((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]))), colI[0], l_run);
+        } else {
+          float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+              asm volatile("" ::: "memory");
+              const float4 iv = *reinterpret_cast<const float4*>(colI + 32 * c + 2 * i);
+              const float p0 = ptx::ex2(__uint_as_float(sr[c][2 * i]) - m_run);
+              const float p1 = ptx::ex2(__uint_as_float(sr[c][2 * i + 1]) - m_run);
+              const float p2 = ptx::ex2(__uint_as_float(sr[c][2 * i + 2]) - m_run);
+              const float p3 = ptx::ex2(__uint_as_float(sr[c][2 * i + 3]) - m_run);
+              pk[i] = ptx::f32x2_to_f16x2(p0, p1);
+              pk[i + 1] = ptx::f32x2_to_f16x2(p2, p3);
+              const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&pk[i]));
+              const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&pk[i + 1]));
+              l4[0] = fmaf(h0.x, iv.x, l4[0]);
+              l4[1] = fmaf(h0.y, iv.y, l4[1]);
+              l4[2] = fmaf(h1.x, iv.z, l4[2]);
+              l4[3] = fmaf(h1.y, iv.w, l4[3]);
+            }
+            ptx::tmem_st16p(tS + 16 * c, pk);
+          }
+          l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        }
+        ptx::tc_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(C::bPFull + 2 * qt + bf));
+      }
+      if (!ok) break;
+      // ---- epilogue: PV of the last sub-tile (and so every MMA of the segment) is complete
+      ok = waitw(bar(C::bODone + 2 * qt + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, p.status);
       if (!ok) break;
       ptx::tc_fence_after();
-      const int ct = j % NCT;
-      const int4 info = *reinterpret_cast<const int4*>(smem + C::oInfo + 16 * ct);
-      const float* colK = reinterpret_cast<const float*>(smem + C::oCol + ct * 2 * BN * 4);
-      const float* colV = colK + BN;
-      const float ck = colK[0] * q_unscale;
-      // A tile inside one chunk with every key valid and a nonzero V scale takes the uniform path
-      // (one logit factor, one cv); any other tile works per column.
-      const bool uni = info.y && colV[0] > 0.0f;
-
-      // The whole 128-column S row: four loads in flight, one wait.
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + 32 * c, sr[c]);
-      ptx::tc_wait_ld_regs(sr[0]);
-      ptx::reg_fence32(sr[1]);
-      ptx::reg_fence32(sr[2]);
-      ptx::reg_fence32(sr[3]);
-
-      // Row maximum of x = S * g_K(chunk) * scale * log2(e) (masked keys -inf).
-      float mx;
-      if (uni) {
-        float m8[8];  // eight independent max chains
-#pragma unroll
-        for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            m8[2 * c] = ptx::fmax3(m8[2 * c], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
-            m8[2 * c + 1] =
-                ptx::fmax3(m8[2 * c + 1], __uint_as_float(sr[c][i + 2]), __uint_as_float(sr[c][i + 3]));
-          }
-        mx = fmaxf(ptx::fmax3(m8[0], m8[1], m8[2]), ptx::fmax3(m8[3], m8[4], ptx::fmax3(m8[5], m8[6], m8[7]))) *
-             ck;
-      } else {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int jj = 32 * c + i;
-            m4[c] = fmaxf(m4[c], jj < info.x ? __uint_as_float(sr[c][i]) * colK[jj] * q_unscale : -INFINITY);
-          }
-        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      }
-      // Lazy rescale: the reference m only moves (to a whole number, so the rescale is an exact
-      // power of two) when the row maximum exceeds it by more than 2^8.  The O rescale uses
-      // warp-collective TMEM accesses, so it runs for the whole warp when any row moved
-      // (alpha = 1 for the rows that did not).
-      const bool grow = mx > m_run + 8.0f;
-      if (__any_sync(0xFFFFFFFFu, grow)) {
-        const float m_new = grow ? ceilf(mx) : m_run;
-        const float alpha = grow ? ptx::ex2(m_run - m_new) : 1.0f;  // 0 while m is -inf
-        l_run *= alpha;
-        m_run = m_new;
-        if (j > 0) {  // O holds tiles < j; PV(j - 1) is complete (it precedes QK(j))
-          ok = waitw(bar(C::bODone + qt), (j - 1) & 1, abort_flag, p.status);
-          if (!ok) break;
-          ptx::tc_fence_after();
-#pragma unroll 1
-          for (int oc = 0; oc < 8; ++oc) {  // 16 columns at a time: the S row stays in registers
-            uint32_t o[16];
-            ptx::tmem_ld16_wait(tO + 16 * oc, o);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            ptx::tmem_st16p(tO + 16 * oc, o);
-          }
-        }
-      }
-
-      // P~ = 2^(x - m) * cv (cv = g_V(chunk) / max g_V), rounded to fp16 pairs and stored over
-      // S's first 64 columns (chunk c -> P columns [16c, 16c + 16)).  The row sum adds the same
-      // rounded values divided by cv, so the rounding largely cancels in O / l; a key of an
-      // all-zero V chunk (cv = 0) adds 0 to O and its p to l.
-      float la = 0.0f, lb = 0.0f;
-      if (uni) {
-        // x = S * ck + log2(cv) - m in packed pairs; eight independent row-sum chains.
-        const float mneg = log2f(colV[0]) - m_run;
-        float l8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) l8[k] = 0.0f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float x0, x1;
-            ptx::ffma2(x0, x1, __uint_as_float(sr[c][2 * i]), __uint_as_float(sr[c][2 * i + 1]), ck, mneg);
-            pk[i] = ptx::f32x2_to_f16x2(ptx::ex2(x0), ptx::ex2(x1));
-            l8[i & 7] = ptx::add_f16x2_f32(l8[i & 7], pk[i]);
-          }
-          ptx::tmem_st16p(tS + 16 * c, pk);
-        }
-        la = (l8[0] + l8[1]) + (l8[2] + l8[3]);
-        lb = (l8[4] + l8[5]) + (l8[6] + l8[7]);
-        l_run += (la + lb) / colV[0];
-      } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int j0 = 32 * c + 2 * i;
-            const float x0 = j0 < info.x ? __uint_as_float(sr[c][2 * i]) * colK[j0] * q_unscale : -INFINITY;
-            const float x1 =
-                j0 + 1 < info.x ? __uint_as_float(sr[c][2 * i + 1]) * colK[j0 + 1] * q_unscale : -INFINITY;
-            const float p0 = x0 == -INFINITY ? 0.0f : ptx::ex2(x0 - m_run);
-            const float p1 = x1 == -INFINITY ? 0.0f : ptx::ex2(x1 - m_run);
-            const float cv0 = colV[j0], cv1 = colV[j0 + 1];
-            pk[i] = ptx::f32x2_to_f16x2(p0 * cv0, p1 * cv1);
-            const float t0 = __half2float(__ushort_as_half(static_cast<uint16_t>(pk[i] & 0xFFFFu)));
-            const float t1 = __half2float(__ushort_as_half(static_cast<uint16_t>(pk[i] >> 16)));
-            la += cv0 > 0.0f ? t0 / cv0 : p0;
-            lb += cv1 > 0.0f ? t1 / cv1 : p1;
-          }
-          ptx::tmem_st16p(tS + 16 * c, pk);
-        }
-        l_run += la + lb;
-      }
-      ptx::tc_wait_st();
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(C::bPFull + qt));
-    }
-    if (ok && p.n_tiles > 0) {
-      ok = waitw(bar(C::bODone + qt), (p.n_tiles - 1) & 1, abort_flag, p.status);
-      if (ok) {
-        ptx::tc_fence_after();
+      ++sq;
+      // Q of this segment is no longer read: load the next segment's Q behind the epilogue.
+      q_pending = issue_q(unext);
+      const int qrow_i = s.m0 + qt * BM + row;
+      const bool store = qrow_i < p.Lq;
+      const bool full = s.t0 == 0 && s.t1 == p.pl.NT;
+      if (full) {
         const float inv = gv_ref / l_run;
-        const int qrow = m0 + qt * BM + row;
-        const bool store = qrow < p.Lq;
-        const int64_t obase = ((static_cast<int64_t>(b) * p.Lq + qrow) * p.H + h) * D;
+        const int64_t obase = ((static_cast<int64_t>(b) * p.Lq + qrow_i) * p.H + h) * D;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
@@ -631,116 +648,211 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
             }
           }
         }
+      } else {
+        // Partial result: unnormalised O, the reference max and the running sum of this range.
+        const int slot = 2 * cta + (u == ubeg ? 0 : 1);
+        float* sp = p.part + static_cast<int64_t>(slot) * kSlotFloats;
+        float4* dst = reinterpret_cast<float4*>(sp + (qt * BM + row) * D);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tO + 32 * c, r);
+          ptx::tc_wait_ld();
+          if (store) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[8 * c + i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                           __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+          }
+        }
+        if (store) {
+          sp[QT * BM * D + qt * BM + row] = m_run;
+          sp[QT * BM * D + QT * BM + qt * BM + row] = l_run;
+        }
+        if (qt == 0 && row == 0) sp[QT * BM * D + 2 * QT * BM] = gv_ref;
       }
+      jjb += ntl;
+      u = unext;
     }
-    }
+    if (!ok && q_pending && issuer) wait_drain(bar(C::bQFull + qt), sq & 1, p.status);
   } else {
-  if constexpr (QT == 2) ptx::setmaxnreg_dec<80>();
-  if (warp == C::kProducerWarp) {
-    // ============================================================ TMA producer
-    if (lane == 0) {
-      ptx::prefetch_tmap(&tmap_q);
-      ptx::mbar_arrive_expect_tx(bar(C::bQFull), nq * TILE16);
-      for (int q = 0; q < nq; ++q)
-        for (int half = 0; half < 2; ++half)
-          ptx::tma_load_4d(sbase + C::oQ + q * TILE16 + half * HALF16, &tmap_q, half * 64, h,
-                           m0 + q * BM, b, bar(C::bQFull));
-      const uint8_t* kc = p.k_codes + bh * p.T * kCodeBytes;
-      const uint8_t* vc = p.v_codes + bh * p.T * kCodeBytes;
-      const uint8_t* ks = p.k_scales + bh * p.T * kScaleBytes;
-      const uint8_t* vs = p.v_scales + bh * p.T * kScaleBytes;
-      int issued = 0;
-      bool ok = true;
-      for (int j = 0; j < p.n_tiles && ok; ++j) {
-        int key0, n;
-        tile_keys(p, j, key0, n);
-        for (int t = 0; t < 2; ++t) {
-          const int pk = 2 * j + t;
-          const int slot = pk % NPK;
-          ok = wait1(bar(C::bPkEmpty + slot), ((pk / NPK) & 1) ^ 1, abort_flag, p.status);
-          if (!ok) break;
-          const uint32_t dst = sbase + C::oPK + slot * PK_BYTES;
-          ptx::mbar_arrive_expect_tx(bar(C::bPkFull + slot), n * (kCodeBytes + kScaleBytes));
-          ptx::bulk_g2s(dst, (t == 0 ? kc : vc) + static_cast<int64_t>(key0) * kCodeBytes,
-                        n * kCodeBytes, bar(C::bPkFull + slot));
-          ptx::bulk_g2s(dst + PK_CODES, (t == 0 ? ks : vs) + static_cast<int64_t>(key0) * kScaleBytes,
-                        n * kScaleBytes, bar(C::bPkFull + slot));
-          issued = pk + 1;
+    ptx::setmaxnreg_dec<88>();
+    if (warp == C::kProducerWarp) {
+      // ========================================================== TMA producer (packed K/V)
+      if (lane == 0) {
+        int issued = 0, pk = 0;
+        bool ok = true;
+        for (int u = ubeg; u < uend && ok;) {
+          const Seg s = plan_seg(p.pl, u, uend);
+          const int64_t bh = s.bhi;
+          const uint8_t* kc = p.k_codes + bh * p.T * kCodeBytes;
+          const uint8_t* vc = p.v_codes + bh * p.T * kCodeBytes;
+          const uint8_t* ks = p.k_scales + bh * p.T * kScaleBytes;
+          const uint8_t* vs = p.v_scales + bh * p.T * kScaleBytes;
+          for (int j = s.t0; j < s.t1 && ok; ++j) {
+            int key0, n;
+            tile_keys(p, j, key0, n);
+            for (int t = 0; t < 2; ++t, ++pk) {
+              const int slot = static_cast<int>(pk % NPK);
+              ok = wait1(bar(C::bPkEmpty + slot), static_cast<uint32_t>((pk / NPK) & 1) ^ 1u, abort_flag, p.status);
+              if (!ok) break;
+              const uint32_t dst = sbase + C::oPK + slot * PK_BYTES;
+              ptx::mbar_arrive_expect_tx(bar(C::bPkFull + slot), n * (kCodeBytes + kScaleBytes));
+              ptx::bulk_g2s(dst, (t == 0 ? kc : vc) + static_cast<int64_t>(key0) * kCodeBytes,
+                            n * kCodeBytes, bar(C::bPkFull + slot));
+              ptx::bulk_g2s(dst + PK_CODES, (t == 0 ? ks : vs) + static_cast<int64_t>(key0) * kScaleBytes,
+                            n * kScaleBytes, bar(C::bPkFull + slot));
+              issued = pk + 1;
+            }
+          }
+          u = seg_end(p.pl, s);
+        }
+        if (!ok) {  // let every copy already issued land before the CTA can exit
+          for (int k = std::max(0, issued - NPK); k < issued; ++k)
+            wait_drain(bar(C::bPkFull + static_cast<int>(k % NPK)), static_cast<uint32_t>((k / NPK) & 1), p.status);
         }
       }
-      if (!ok) {  // let every copy already issued land before the CTA can exit
-        wait_drain(bar(C::bQFull), 0, p.status);
-        for (int pk = std::max(0, issued - NPK); pk < issued; ++pk)
-          wait_drain(bar(C::bPkFull + pk % NPK), (pk / NPK) & 1, p.status);
-      }
-    }
-    __syncwarp();
-  } else if (warp == C::kMmaWarp) {
-    // ============================================================ MMA issuer
-    // The whole warp runs this loop with warp-uniform values; one elected lane issues each
-    // tcgen05 instruction.
-    // kind::f16 instruction descriptors: fp16 x fp16 -> fp32; M = 128; N = 128.
-    constexpr uint32_t kIdescQK = (1u << 4) |  // A = Q and B = K^ both K-major
-                                  (static_cast<uint32_t>(BN >> 3) << 17) |
-                                  (static_cast<uint32_t>(BM >> 4) << 24);
-    constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) |  // B = V^ MN-major
-                                  (static_cast<uint32_t>(D >> 3) << 17) |
-                                  (static_cast<uint32_t>(BM >> 4) << 24);
-    // Shared-memory descriptors are built once; a K step only advances the 14-bit start address
-    // field (address >> 4).
-    const uint64_t dQ0 = ptx::smem_desc_sw128(sbase + C::oQ, 16, 1024);
-    const uint64_t dK0 = ptx::smem_desc_sw128(sbase + C::oK, 16, 1024);
-    const uint64_t dV0 = ptx::smem_desc_sw128(sbase + C::oV, HALF16, 1024);
-    auto issue_qk = [&](int q, int st) {
-      const uint64_t dQ = dQ0 + static_cast<uint64_t>((q * TILE16) >> 4);
-      const uint64_t dK = dK0 + static_cast<uint64_t>((st * TILE16) >> 4);
-      const uint32_t tS = tmem + q * BN;
-      // one asm block of eight MMAs: a rolled loop issued an MMA only every ~80 cycles
-      ptx::mma_qk8_w(tS, dQ, dK, kIdescQK, 0u);
-      ptx::mma_commit_w(bar(C::bSFull + q));
-    };
-    bool ok = waitw(bar(C::bQReady), 0, abort_flag, p.status) && p.n_tiles > 0 &&
-              waitw(bar(C::bKFull + 0), 0, abort_flag, p.status);
-    if (ok) {
-      ptx::tc_fence_after();
-      for (int q = 0; q < nq; ++q) issue_qk(q, 0);
-      ptx::mma_commit_w(bar(C::bKEmpty + 0));
-    }
-    // Per KV tile j: PV(q, j) as soon as softmax q has written P(q, j), then QK(q, j + 1) into the
-    // same S columns; the two query tiles alternate so the tensor core always has the other
-    // tile's work while one softmax runs.
-    for (int j = 0; j < p.n_tiles && ok; ++j) {
-      const int st = j % NST;
-      for (int q = 0; q < nq && ok; ++q) {
-        ok = waitw(bar(C::bPFull + q), j & 1, abort_flag, p.status);
-        if (ok && q == 0) ok = waitw(bar(C::bVFull + st), (j / NST) & 1, abort_flag, p.status);
+      __syncwarp();
+    } else if (warp == C::kMmaWarp) {
+      // ========================================================== MMA issuer
+      // The whole warp runs this loop with warp-uniform values; one elected lane issues each
+      // tcgen05 instruction.  kind::f16 instruction descriptors: fp16 x fp16 -> fp32; M = 128.
+      constexpr uint32_t kIdescQK = (1u << 4) |  // A = Q and B = K^ both K-major; N = 64 keys
+                                    (static_cast<uint32_t>(SUB >> 3) << 17) |
+                                    (static_cast<uint32_t>(BM >> 4) << 24);
+      constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) |  // B = V^ MN-major; N = 128 dims
+                                    (static_cast<uint32_t>(D >> 3) << 17) |
+                                    (static_cast<uint32_t>(BM >> 4) << 24);
+      // Shared-memory descriptors are built once; a step only advances the 14-bit start address
+      // field (address >> 4).  Sub-tile `half` of a K or V stage starts 64 rows (8 KB) in.
+      const uint64_t dQ0 = ptx::smem_desc_sw128(sbase + C::oQ, 16, 1024);
+      const uint64_t dK0 = ptx::smem_desc_sw128(sbase + C::oK, 16, 1024);
+      const uint64_t dV0 = ptx::smem_desc_sw128(sbase + C::oV, HALF16, 1024);
+      auto issue_qk = [&](int q, int bf, int st, int half) {
+        const uint64_t dQ = dQ0 + static_cast<uint64_t>((q * TILE16) >> 4);
+        const uint64_t dK = dK0 + static_cast<uint64_t>((st * TILE16 + half * SUB * 128) >> 4);
+        ptx::mma_qk8_w(tmem + (2 * q + bf) * SUB, dQ, dK, kIdescQK, 0u);
+        ptx::mma_commit_w(bar(C::bSFull + 2 * q + bf));
+      };
+      auto issue_pv = [&](int q, int bf, int st, int half, uint32_t acc) {
+        const uint64_t dV = dV0 + static_cast<uint64_t>((st * TILE16 + half * SUB * 128) >> 4);
+        ptx::mma_pv4_w(tmem + C::kTmemO + q * D, tmem + (2 * q + bf) * SUB, dV, kIdescPV, acc);
+        ptx::mma_commit_w(bar(C::bODone + 2 * q + bf));
+      };
+      int gq[QT] = {0, 0}, sq[QT] = {0, 0};
+      int jjb = 0;
+      bool ok = true;
+      for (int u = ubeg; u < uend && ok;) {
+        const Seg s = plan_seg(p.pl, u, uend);
+        const int ntl = s.t1 - s.t0, nq = s.nq, nh = 2 * ntl;
+        for (int q = 0; q < nq && ok; ++q) ok = waitw(bar(C::bQReady + q), sq[q] & 1, abort_flag, p.status);
+        const int st0 = static_cast<int>(jjb % NST);
+        if (ok) ok = waitw(bar(C::bKFull + st0), static_cast<uint32_t>((jjb / NST) & 1), abort_flag, p.status);
         if (!ok) break;
         ptx::tc_fence_after();
-        const uint64_t dV = dV0 + static_cast<uint64_t>((st * TILE16) >> 4);
-        const uint32_t tO = tmem + QT * BN + q * D, tP = tmem + q * BN;
-        ptx::mma_pv8_w(tO, tP, dV, kIdescPV, j > 0 ? 1u : 0u);
-        ptx::mma_commit_w(bar(C::bODone + q));
-        if (q == nq - 1) ptx::mma_commit_w(bar(C::bVEmpty + st));
-        if (j + 1 < p.n_tiles) {
-          const int st1 = (j + 1) % NST;
-          if (q == 0) {
-            ok = waitw(bar(C::bKFull + st1), ((j + 1) / NST) & 1, abort_flag, p.status);
+        // both sub-tiles of the segment's first KV tile, for every query tile
+        for (int q = 0; q < nq; ++q)
+          for (int hs = 0; hs < 2; ++hs) issue_qk(q, (gq[q] + hs) & 1, st0, hs);
+        ptx::mma_commit_w(bar(C::bKEmpty + st0));
+        // Per sub-tile hs: PV(q, hs) as soon as softmax q has written P(q, hs), then QK(q, hs + 2)
+        // into the same S buffer; the two query tiles alternate.
+        for (int hs = 0; hs < nh && ok; ++hs) {
+          const int jt = jjb + (hs >> 1);
+          const int st = static_cast<int>(jt % NST), half = hs & 1;
+          for (int q = 0; q < nq; ++q) {
+            const int gg = gq[q] + hs, bf = gg & 1;
+            ok = waitw(bar(C::bPFull + 2 * q + bf), (gg >> 1) & 1, abort_flag, p.status);
+            if (ok && q == 0 && half == 0) ok = waitw(bar(C::bVFull + st), static_cast<uint32_t>((jt / NST) & 1), abort_flag, p.status);
             if (!ok) break;
             ptx::tc_fence_after();
+            issue_pv(q, bf, st, half, hs > 0 ? 1u : 0u);
+            if (q == nq - 1 && half == 1) ptx::mma_commit_w(bar(C::bVEmpty + st));
+            if (hs + 2 < nh) {
+              const int jt2 = jjb + ((hs + 2) >> 1);
+              const int st2 = static_cast<int>(jt2 % NST);
+              if (q == 0 && half == 0) {
+                ok = waitw(bar(C::bKFull + st2), static_cast<uint32_t>((jt2 / NST) & 1), abort_flag, p.status);
+                if (!ok) break;
+                ptx::tc_fence_after();
+              }
+              issue_qk(q, bf, st2, half);
+              if (q == nq - 1 && half == 1) ptx::mma_commit_w(bar(C::bKEmpty + st2));
+            }
           }
-          issue_qk(q, st1);
-          if (q == nq - 1) ptx::mma_commit_w(bar(C::bKEmpty + st1));
         }
+        for (int q = 0; q < nq; ++q) {
+          gq[q] += nh;
+          ++sq[q];
+        }
+        jjb += ntl;
+        u = seg_end(p.pl, s);
+      }
+      // every MMA issued so far completes before the drain barrier's phase 0
+      ptx::mma_commit_w(bar(C::bDrain));
+      if (lane == 0) wait_drain(bar(C::bDrain), 0, p.status);
+      __syncwarp();
+    } else {
+      // ========================================================== dequant warps
+      // No barrier among the dequant warps: each works through the same tiles on its own, so a
+      // warp that gives up after a time-out never leaves the others waiting.
+      const int dt = threadIdx.x - C::kDequantWarp0 * 32;
+      float inv_gv = 1.0f;
+      int jj = 0;
+      bool ok = true;
+      for (int u = ubeg; u < uend && ok;) {
+        const Seg s = plan_seg(p.pl, u, uend);
+        const int64_t bh = s.bhi;
+        inv_gv = 1.0f / max_visible_gv(p, bh);
+        for (int j = s.t0; j < s.t1 && ok; ++j, ++jj) {
+          const int st = static_cast<int>(jj % NST);
+          int key0, n;
+          tile_keys(p, j, key0, n);
+          // The FP32 scales of this thread's key for the per-column tables, loaded before the waits.
+          float gk = 0.0f, gvv = 0.0f;
+          if (dt < n) {
+            const int64_t c = bh * p.C + (key0 + dt) / p.Lc;
+            gk = p.k_g[c] * p.scale_log2;
+            gvv = p.v_g[c] * inv_gv;
+            if (!(gvv > 0.0f)) gvv = 1.0f;  // an all-zero V chunk: V^ rows are 0, P only counts in l
+          }
+          for (int t = 0; t < 2 && ok; ++t) {
+            // the stage's previous tile (jj - NST) is done with it: K after its QKs, V after its PVs
+            if (jj >= NST)
+              ok = waitw(bar((t == 0 ? C::bKEmpty : C::bVEmpty) + st), static_cast<uint32_t>(((jj / NST) - 1) & 1),
+                         abort_flag, p.status);
+            if (!ok) break;
+            const int pk = 2 * jj + t;
+            const int slot = static_cast<int>(pk % NPK);
+            ok = waitw(bar(C::bPkFull + slot), static_cast<uint32_t>((pk / NPK) & 1), abort_flag, p.status);
+            if (!ok) break;
+            const uint8_t* src = smem + C::oPK + slot * PK_BYTES;
+            uint8_t* dst = smem + (t == 0 ? C::oK : C::oV) + st * TILE16;
+            if (n == BN) dequant_tile<C::kDequantThreads, true>(src, dst, n, dt);
+            else dequant_tile<C::kDequantThreads, false>(src, dst, n, dt);
+            if (t == 0 && dt < BN) {  // per-column tables: one thread per key of the tile
+              const int ct = static_cast<int>(jj % NCT);
+              float* colK = reinterpret_cast<float*>(smem + C::oCol + ct * C::kColTab);
+              const bool valid = dt < n;
+              colK[dt] = gk;
+              colK[BN + dt] = valid ? __log2f(gvv) : -INFINITY;
+              colK[2 * BN + dt] = valid ? __frcp_rn(gvv) : 0.0f;
+              if (dt == 0) {
+                const int uniform = (n == BN) && (key0 / p.Lc == (key0 + BN - 1) / p.Lc);
+                *reinterpret_cast<int4*>(smem + C::oInfo + 16 * ct) = make_int4(n, uniform, 0, 0);
+              }
+            }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              ptx::mbar_arrive(bar(C::bPkEmpty + slot));
+              ptx::mbar_arrive(bar(t == 0 ? C::bKFull + st : C::bVFull + st));
+              if (t == 0) ptx::mbar_arrive(bar(C::bTabFull + static_cast<int>(jj % NCT)));
+            }
+          }
+        }
+        u = seg_end(p.pl, s);
       }
     }
-    // every MMA issued so far completes before the drain barrier's phase 0
-    ptx::mma_commit_w(bar(C::bDrain));
-    if (lane == 0) wait_drain(bar(C::bDrain), 0, p.status);
-    __syncwarp();
-  } else {
-    // ============================================================ dequant warps
-    dequant_role(threadIdx.x - C::kDequantWarp0 * 32);
-  }
   }
 
   ptx::tc_fence_before();
@@ -748,6 +860,71 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
   if (warp == C::kMmaWarp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// Merges the partial results of every work item whose KV tiles were split between CTAs.  Block
+// b - 1 looks at the boundary between CTAs b - 1 and b; the first boundary inside an item merges
+// that item.  One warp per query row: each lane owns 4 of the 128 columns.
+//   m* = max_k m_k;  O = sum_k O_k 2^(m_k - m*);  l = sum_k l_k 2^(m_k - m*);  out = O g_ref / l
+// (the m_k are whole numbers, so every factor is an exact power of two).
+__global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ AttnParams p) {
+  const Plan& pl = p.pl;
+  const int bnd = blockIdx.x + 1;
+  const int64_t u = plan_cut(pl, bnd);
+  if (u >= pl.units || u % pl.NT == 0) return;
+  const int64_t item = u / pl.NT, istart = item * pl.NT, iend = istart + pl.NT;
+  if (plan_cut(pl, bnd - 1) > istart) return;  // an earlier boundary lies inside this item
+  __shared__ int slots[kMaxCtas];
+  __shared__ int n_slots;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int c = bnd - 1; c < pl.G; ++c) {
+      const int64_t cs = plan_cut(pl, c), ce = plan_cut(pl, c + 1);
+      if (cs >= iend) break;
+      if (ce <= istart || cs == ce) continue;
+      slots[n++] = 2 * c + (cs < istart ? 1 : 0);
+    }
+    n_slots = n;
+  }
+  __syncthreads();
+  const int ns = n_slots;
+  const int bhi = static_cast<int>(item / pl.ipb), k = static_cast<int>(item % pl.ipb);
+  const int m0 = 2 * k * BM, nq = (2 * k + 1 < pl.n_qt) ? 2 : 1;
+  const int b = bhi / p.H, h = bhi % p.H;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float gv = p.part[static_cast<int64_t>(slots[0]) * kSlotFloats + QT * BM * D + 2 * QT * BM];
+  for (int r = warp; r < nq * BM; r += 8) {
+    const int qrow = m0 + r;
+    if (qrow >= p.Lq) continue;
+    float mstar = -INFINITY;
+    for (int i = 0; i < ns; ++i)
+      mstar = fmaxf(mstar, p.part[static_cast<int64_t>(slots[i]) * kSlotFloats + QT * BM * D + r]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float l = 0.0f;
+    for (int i = 0; i < ns; ++i) {
+      const float* sp = p.part + static_cast<int64_t>(slots[i]) * kSlotFloats;
+      const float wgt = ptx::ex2(sp[QT * BM * D + r] - mstar);
+      const float4 o = reinterpret_cast<const float4*>(sp + r * D)[lane];
+      acc.x += wgt * o.x;
+      acc.y += wgt * o.y;
+      acc.z += wgt * o.z;
+      acc.w += wgt * o.w;
+      l += wgt * sp[QT * BM * D + QT * BM + r];
+    }
+    const float inv = gv / l;
+    const int64_t obase = ((static_cast<int64_t>(b) * p.Lq + qrow) * p.H + h) * D + 4 * lane;
+    if (p.out_bf16) {
+      __nv_bfloat162 v0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      __nv_bfloat162 v1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+      uint2 w;
+      w.x = *reinterpret_cast<uint32_t*>(&v0);
+      w.y = *reinterpret_cast<uint32_t*>(&v1);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + obase) = w;
+    } else {
+      *reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase) =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
   }
 }
 
@@ -767,82 +944,49 @@ __global__ void __launch_bounds__(32) wait_timeout_probe(uint32_t* status) {
 }
 
 // ------------------------------------------------------------------ host side
-template <int QT>
-cudaError_t launch(const CUtensorMap& tm, const AttnParams& prm, int n_single_ctas, cudaStream_t stream) {
-  using C = Cfg<QT>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(attention_kernel<QT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    C::kSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
-  attention_kernel<QT><<<prm.n_pair_ctas + n_single_ctas, C::kThreads, C::kSmemBytes, stream>>>(tm, prm);
-  return cudaGetLastError();
+PerDeviceOnce g_attn_attr;
+
+// The work split for bh (batch, head) pairs of n_qt query tiles over NT KV tiles on n_sms SMs.
+Plan make_plan(int64_t bh, int n_qt, int NT, int n_sms) {
+  Plan pl{};
+  pl.bh = static_cast<int>(bh);
+  pl.n_qt = n_qt;
+  pl.ipb = (n_qt + 1) / 2;
+  pl.npairs = n_qt / 2;
+  pl.NT = NT;
+  pl.wP = kWPair;
+  pl.wS = kWSingle;
+  pl.units = bh * pl.ipb * static_cast<int64_t>(NT);
+  pl.Wh = static_cast<int64_t>(NT) * (static_cast<int64_t>(pl.wP) * pl.npairs +
+                                      static_cast<int64_t>(pl.wS) * (pl.ipb - pl.npairs));
+  pl.W = bh * pl.Wh;
+  // one CTA per SM, at least two KV tiles of work each
+  int64_t g = std::min<int64_t>(std::min(n_sms, kMaxCtas), std::max<int64_t>(1, pl.units / 2));
+  pl.G = static_cast<int>(std::max<int64_t>(1, g));
+  return pl;
 }
 
-// Makespan of p two-tile CTAs (cost `pair`) followed by s one-tile CTAs (cost `single`), each
-// started on whichever of the g SMs frees first (one CTA per SM at a time).  Integer costs keep
-// equal loads equal; machines are tracked per load level, so the cost is the number of levels the
-// schedule passes through, not the number of CTAs.
-int64_t makespan(int64_t p, int64_t s, int64_t g, int64_t pair, int64_t single) {
-  std::map<int64_t, int64_t> level;  // load -> machines at that load
-  level[(p / g) * pair] += g - p % g;
-  if (p % g) level[(p / g + 1) * pair] += p % g;
-  while (s > 0) {
-    auto lo = level.begin();
-    const int64_t take = std::min(lo->second, s);
-    const int64_t load = lo->first;
-    s -= take;
-    if ((lo->second -= take) == 0) level.erase(lo);
-    level[load + single] += take;
+bool plan_has_splits(const Plan& pl) {
+  for (int c = 1; c < pl.G; ++c) {
+    const int64_t u = plan_cut(pl, c);
+    if (u < pl.units && u % pl.NT != 0) return true;
   }
-  return level.rbegin()->first;
+  return false;
 }
 
-// Splits the n_qt query tiles of each of the bh (batch, head) pairs into tile pairs (two-tile CTAs,
-// the two softmax warpgroups in ping-pong) and single tiles (one-tile CTAs) so that the launch
-// finishes soonest on g SMs: e.g. 444 tiles on 148 SMs as 148 pairs + 148 singles (1.94 units)
-// instead of 222 pairs in two waves (2 units).  Candidates: all pairs, no pairs, and the last
-// three whole waves of pairs.  Plans are cached per (n_qt, bh, g).
-void plan_work(int n_qt, int bh, int g, AttnParams& prm, int& n_single_ctas) {
-  // Cost of a one-tile CTA relative to a two-tile one (94 : 100), measured on the 1.3B-class
-  // layer: the per-KV-tile dequantisation and MMA chain, which do not shrink with one query tile,
-  // dominate.
-  constexpr int64_t kPair = 100, kSingle = 94;
-  static std::mutex mu;
-  static std::map<std::tuple<int, int, int>, int> cache;
-  int best_p = -1;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    auto it = cache.find(std::make_tuple(n_qt, bh, g));
-    if (it != cache.end()) best_p = it->second;
-  }
-  const int64_t max_p = static_cast<int64_t>(bh) * (n_qt / 2), total = static_cast<int64_t>(bh) * n_qt;
-  if (best_p < 0) {
-    std::vector<int64_t> cand = {0, max_p};
-    for (int64_t k = max_p / g; k >= 1 && k >= max_p / g - 2; --k) cand.push_back(k * g);
-    int64_t bp = max_p, best = makespan(max_p, total - 2 * max_p, g, kPair, kSingle);
-    for (int64_t pc : cand) {
-      const int64_t m = makespan(pc, total - 2 * pc, g, kPair, kSingle);
-      if (m < best || (m == best && pc > bp)) {
-        best = m;
-        bp = pc;
-      }
-    }
-    best_p = static_cast<int>(bp);
-    std::lock_guard<std::mutex> lock(mu);
-    if (cache.size() > 4096) cache.clear();
-    cache[std::make_tuple(n_qt, bh, g)] = best_p;
-  }
-  prm.n_qt = n_qt;
-  prm.pp = best_p / bh;
-  prm.pr = best_p % bh;
-  prm.n_pair_ctas = best_p;
-  n_single_ctas = static_cast<int>(total - 2 * best_p);
-}
+size_t slot_bytes() { return static_cast<size_t>(kSlotFloats) * sizeof(float); }
 
 }  // namespace
+
+int current_sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return sms;
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -858,26 +1002,52 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-size_t attention_workspace_bytes(const nvfp4kv_cache&, int) { return 0; }
+// Two partial-result slots per CTA, one CTA per SM of the current device (148 when no device
+// can be queried).
+size_t attention_workspace_bytes(const nvfp4kv_cache&, int) {
+  int sms = current_sm_count();
+  if (sms <= 0) sms = 148;
+  return 2 * static_cast<size_t>(std::min(sms, kMaxCtas)) * slot_bytes();
+}
+
+bool attention_shape_supported(const nvfp4kv_cache& c, int q_tokens, int64_t kv_tiles) {
+  const int64_t bh = static_cast<int64_t>(c.batch) * c.heads;
+  const int64_t ipb = ((q_tokens + BM - 1) / BM + 1) / 2;
+  // weighted unit arithmetic stays far below 2^62
+  return kv_tiles > 0 && kv_tiles < (int64_t(1) << 24) &&
+         static_cast<double>(bh) * ipb * kv_tiles < 2147483647.0;
+}
 
 cudaError_t launch_wait_timeout_probe(uint32_t* status, cudaStream_t stream) {
   wait_timeout_probe<<<1, 32, 0, stream>>>(status);
   return cudaGetLastError();
 }
 
-int attention_plan(const nvfp4kv_cache& c, int q_tokens, int n_sms, int cta, int out[4]) {
-  AttnParams prm{};
-  int n_single = 0;
+int attention_plan(const nvfp4kv_cache& c, int q_tokens, int kv_tiles, int n_sms, int cta, int seg,
+                   int out[8]) {
+  for (int i = 0; i < 8; ++i) out[i] = 0;
   const int n_qt = (q_tokens + BM - 1) / BM;
-  plan_work(n_qt, c.batch * c.heads, n_sms, prm, n_single);
-  out[0] = prm.n_pair_ctas + n_single;
-  out[1] = out[2] = out[3] = 0;
+  const Plan pl = make_plan(static_cast<int64_t>(c.batch) * c.heads, n_qt, kv_tiles, n_sms);
+  out[0] = pl.G;
+  out[1] = plan_has_splits(pl) ? 2 : 1;
   if (cta < 0) return NVFP4KV_OK;
-  if (cta >= out[0]) return NVFP4KV_ERR_INVALID_ARG;
-  const WorkItem w = work_item(cta, prm.n_qt, prm.pp, prm.pr, prm.n_pair_ctas);
-  out[1] = w.bhi;
-  out[2] = w.m0;
-  out[3] = w.nq;
+  if (cta >= pl.G) return NVFP4KV_ERR_INVALID_ARG;
+  const int64_t ubeg = plan_cut(pl, cta), uend = plan_cut(pl, cta + 1);
+  int n = 0;
+  for (int u = static_cast<int>(ubeg); u < static_cast<int>(uend); ++n) {
+    const Seg s = plan_seg(pl, u, static_cast<int>(uend));
+    if (n == seg) {
+      out[2] = s.bhi;
+      out[3] = s.m0;
+      out[4] = s.nq;
+      out[5] = s.t0;
+      out[6] = s.t1;
+      out[7] = (s.t0 == 0 && s.t1 == pl.NT) ? -1 : 2 * cta + (u == ubeg ? 0 : 1);
+    }
+    u = seg_end(pl, s);
+  }
+  out[1] = n;  // segments of this CTA
+  if (seg >= n) return seg < 0 ? NVFP4KV_OK : NVFP4KV_ERR_INVALID_ARG;
   return NVFP4KV_OK;
 }
 
@@ -889,8 +1059,8 @@ int attention_runs(const std::vector<int>& vis) {
 }
 
 int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, int64_t q_stride,
-                     const std::vector<int>& vis, float softmax_scale, void* out, int out_dtype, void*,
-                     size_t, cudaStream_t stream) {
+                     const std::vector<int>& vis, float softmax_scale, void* out, int out_dtype,
+                     void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   AttnParams prm{};
   prm.k_codes = c.k_codes;
   prm.v_codes = c.v_codes;
@@ -899,6 +1069,7 @@ int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, in
   prm.k_g = c.k_gscale;
   prm.v_g = c.v_gscale;
   prm.out = out;
+  prm.part = static_cast<float*>(workspace);
   prm.status = c.status;
   prm.T = static_cast<int64_t>(c.capacity_chunks) * c.chunk_tokens;
   prm.B = c.batch;
@@ -925,6 +1096,7 @@ int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, in
     i = k + 1;
   }
   prm.n_tiles = prm.run_tile0[prm.n_runs];
+  if (!attention_shape_supported(c, q_tokens, prm.n_tiles)) return NVFP4KV_ERR_UNSUPPORTED;
 
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return NVFP4KV_ERR_CUDA;
@@ -939,14 +1111,24 @@ int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, in
                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return NVFP4KV_ERR_CUDA;
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return NVFP4KV_ERR_CUDA;
-  int n_single_ctas = 0;
-  plan_work((q_tokens + BM - 1) / BM, c.batch * c.heads, sms, prm, n_single_ctas);
-  const cudaError_t e = launch<2>(tm, prm, n_single_ctas, stream);
-  return e == cudaSuccess ? NVFP4KV_OK : NVFP4KV_ERR_CUDA;
+  const int sms = current_sm_count();
+  if (sms <= 0) return NVFP4KV_ERR_CUDA;
+  prm.pl = make_plan(static_cast<int64_t>(c.batch) * c.heads, (q_tokens + BM - 1) / BM, prm.n_tiles, sms);
+  const bool splits = plan_has_splits(prm.pl);
+  if (splits && (!workspace || workspace_bytes < 2 * static_cast<size_t>(prm.pl.G) * slot_bytes()))
+    return NVFP4KV_ERR_WORKSPACE;
+
+  const cudaError_t ae = g_attn_attr.run([] {
+    return cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+  });
+  if (ae != cudaSuccess) return NVFP4KV_ERR_CUDA;
+  attention_kernel<<<prm.pl.G, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tm, prm);
+  if (cudaGetLastError() != cudaSuccess) return NVFP4KV_ERR_CUDA;
+  if (splits) {
+    combine_kernel<<<prm.pl.G - 1, 256, 0, stream>>>(prm);
+    if (cudaGetLastError() != cudaSuccess) return NVFP4KV_ERR_CUDA;
+  }
+  return NVFP4KV_OK;
 }
 
 }  // namespace nvfp4kv

@@ -4,8 +4,11 @@
 // Dequantisation follows the "LongLive-2.0" reading note, "The NVFP4 quantization format":
 // x_hat = (E2M1 element) * (E4M3 block scale) * (FP32 scale).  The first product is formed
 // exactly in 16-bit floating point with the same helpers the attention kernel uses for its
-// in-shared-memory dequantisation (bf16 for K, fp16 for V), then multiplied by the FP32
-// scale with a single fp32 rounding.
+// in-shared-memory dequantisation (exact code * scale products), then multiplied by the FP32
+// scale with a single fp32 rounding.  (Both 16-bit forms hold the product exactly; the attention
+// kernel stages K and V as fp16.)
+#include <algorithm>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -75,8 +78,8 @@ cudaError_t launch_dequantize(const nvfp4kv_cache& c, int which, int first_slot,
   const bool is_k = which == 0;
   const int BH = c.batch * c.heads;
   const int64_t total = static_cast<int64_t>(BH) * n_slots * c.chunk_tokens * 16;
-  int blocks = static_cast<int>((total + 255) / 256);
-  if (blocks > 148 * 16) blocks = 148 * 16;
+  const int sms = current_sm_count();
+  int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 16 * static_cast<int64_t>(sms > 0 ? sms : 1)));
   if (blocks < 1) blocks = 1;
   dequant_kernel<<<blocks, 256, 0, stream>>>(is_k ? c.k_codes : c.v_codes,
                                              is_k ? c.k_scales : c.v_scales,
@@ -88,8 +91,8 @@ cudaError_t launch_dequantize(const nvfp4kv_cache& c, int which, int first_slot,
 
 cudaError_t launch_encode_probe(const float* x, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
                                 cudaStream_t stream) {
-  int blocks = static_cast<int>((n + 255) / 256);
-  if (blocks > 148 * 32) blocks = 148 * 32;
+  const int sms = current_sm_count();
+  int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, 32 * static_cast<int64_t>(sms > 0 ? sms : 1)));
   if (blocks < 1) blocks = 1;
   encode_probe_kernel<<<blocks, 256, 0, stream>>>(x, n, e2m1, e4m3);
   return cudaGetLastError();

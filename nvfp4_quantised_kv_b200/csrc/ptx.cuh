@@ -243,6 +243,25 @@ __device__ __forceinline__ void mma_pv8_w(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+//   PV form over 64 keys: four K = 16 steps (A: 8 TMEM columns per step; B: 2048 B per step).
+__device__ __forceinline__ void mma_pv4_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t.reg .b32 blo, bhi, t1, ta;\n\t.reg .b64 db;\n\t"
+      "mov.b64 {blo, bhi}, %2;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.s32 ta, %1, 8;\n\tadd.s32 t1, blo, 128;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 16;\n\tadd.s32 t1, blo, 256;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 24;\n\tadd.s32 t1, blo, 384;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"

@@ -99,14 +99,9 @@ __device__ __forceinline__ Encoder make_encoder(float g, float* rtab, int tid, i
   return e;
 }
 
-// Encodes this lane's 8 elements of a 16-element block (its partner lane xor 1 holds the other 8)
-// and stores the 4 code bytes and, from the even lane, the scale byte.
-__device__ __forceinline__ void encode_store(uint4 w, const Encoder& e, const float* rtab, bool valid,
-                                             uint8_t* code_dst, uint8_t* scale_dst, int lane) {
-  uint32_t mb = absmax_bits(w);
-  mb = max(mb & 0xFFFFu, mb >> 16);
-  mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 1));
-  const float ab = __uint_as_float(mb << 16);
+// E4M3 code of the block scale s = RN_e4m3(a_b / (6 g)) for the block maximum a_b (0 when a_b or
+// g is 0).
+__device__ __forceinline__ uint32_t block_scale_code(float ab, const Encoder& e) {
   uint32_t s_code = 0;
   if (ab != 0.0f && e.g != 0.0f) {
     float q;
@@ -119,22 +114,54 @@ __device__ __forceinline__ void encode_store(uint4 w, const Encoder& e, const fl
     }
     s_code = ptx::f32_to_e4m3(q);
   }
-  const float r = rtab[s_code & 0x7F];
-  uint32_t qc = 0;
-  if (r != 0.0f) {
-    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-    float y[8];
+  return s_code;
+}
+
+// E2M1 codes of 8 bf16 elements (one 16-byte word) times r, element 2j in the low nibble of
+// byte j; 0 when r is 0.
+__device__ __forceinline__ uint32_t codes8(uint4 w, float r) {
+  if (r == 0.0f) return 0u;
+  const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+  float y[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      y[2 * i] = __fmul_rn(__uint_as_float(wv[i] << 16), r);
-      y[2 * i + 1] = __fmul_rn(__uint_as_float(wv[i] & 0xFFFF0000u), r);
-    }
-    qc = ptx::f32x8_to_e2m1x8(y);
+  for (int i = 0; i < 4; ++i) {
+    y[2 * i] = __fmul_rn(__uint_as_float(wv[i] << 16), r);
+    y[2 * i + 1] = __fmul_rn(__uint_as_float(wv[i] & 0xFFFF0000u), r);
   }
+  return ptx::f32x8_to_e2m1x8(y);
+}
+
+// Encodes this lane's 8 elements of a 16-element block (its partner lane xor 1 holds the other 8)
+// and stores the 4 code bytes and, from the even lane, the scale byte.
+__device__ __forceinline__ void encode_store(uint4 w, const Encoder& e, const float* rtab, bool valid,
+                                             uint8_t* code_dst, uint8_t* scale_dst, int lane) {
+  uint32_t mb = absmax_bits(w);
+  mb = max(mb & 0xFFFFu, mb >> 16);
+  mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 1));
+  const uint32_t s_code = block_scale_code(__uint_as_float(mb << 16), e);
+  const uint32_t qc = codes8(w, rtab[s_code & 0x7F]);
   if (valid) {
     *reinterpret_cast<uint32_t*>(code_dst) = qc;
     if ((lane & 1) == 0) *scale_dst = static_cast<uint8_t>(s_code);
   }
+}
+
+// Encodes 32 consecutive elements of one token row (blocks 2j and 2j + 1, four 16-byte words)
+// and stores their 16 code bytes and 2 scale bytes with one 16-byte and one 2-byte store.
+__device__ __forceinline__ void encode32_store(const uint4 (&w)[4], const Encoder& e, const float* rtab,
+                                               uint8_t* code_dst, uint8_t* scale_dst) {
+  uint32_t qc[4], sc[2];
+#pragma unroll
+  for (int blk = 0; blk < 2; ++blk) {
+    uint32_t mb = __vmaxu2(absmax_bits(w[2 * blk]), absmax_bits(w[2 * blk + 1]));
+    mb = max(mb & 0xFFFFu, mb >> 16);
+    sc[blk] = block_scale_code(__uint_as_float(mb << 16), e);
+    const float r = rtab[sc[blk] & 0x7F];
+    qc[2 * blk] = codes8(w[2 * blk], r);
+    qc[2 * blk + 1] = codes8(w[2 * blk + 1], r);
+  }
+  *reinterpret_cast<uint4*>(code_dst) = make_uint4(qc[0], qc[1], qc[2], qc[3]);
+  *reinterpret_cast<uint16_t*>(scale_dst) = static_cast<uint16_t>(sc[0] | (sc[1] << 8));
 }
 
 __global__ void __launch_bounds__(kThreads, 6) amax_kernel(const __grid_constant__ QuantArgs a) {
@@ -216,6 +243,138 @@ __global__ void __launch_bounds__(kThreads, 6) quantize_kernel(const __grid_cons
     const int t = t_begin + u * (kThreads / 16) + sub;
     encode_store(w[u], enc, rtab, t < t_end, codes + static_cast<int64_t>(t) * kCodeBytes,
                  scales + static_cast<int64_t>(t) * kScaleBytes, lane);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Single-launch path for one or many layers (ticketed).  A slice is one (layer, tensor, b, h) of
+// the new chunk; a part is kTicketTokens of its tokens.  Every CTA takes a ticket t in the order
+// CTAs start (an atomic counter) and
+//   1. reduces max|x| over part t and folds it into its slice's maximum (atomicMax on the bf16
+//      magnitude bits), then counts the part as done;
+//   2. encodes part e = t - lag once every part of e's slice is done, re-reading its rows (still in
+//      L2: at most about lag parts were read since).
+// Step 2 only waits for tickets below t, which belong to CTAs that already started and whose
+// step 1 waits for nothing, so the wait always ends; it is still bounded (the status bit is set
+// if it ever runs out).  The input crosses HBM once for any number of layers.
+constexpr int kMaxLayers = 64;
+constexpr int kTicketTokens = 128;
+
+struct TicketArgs {
+  const uint16_t* x[kMaxLayers][2];
+  uint8_t* codes[kMaxLayers][2];
+  uint8_t* scales[kMaxLayers][2];
+  float* gscale[kMaxLayers][2];
+  uint32_t* ctr;  // [0] ticket counter; per slice s: [1 + 2s] max|x| bits, [2 + 2s] parts done
+  uint32_t* status;
+  int64_t token_stride;
+  int64_t T;  // tokens per (b, h) in the cache
+  int B, H, L, C, slot, parts, lag;
+  int n_work;  // slices * parts
+};
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(kThreads, 4) quantize_ticket_kernel(const __grid_constant__ TicketArgs a) {
+  __shared__ int s_ticket;
+  __shared__ uint32_t red[kWarps];
+  __shared__ float s_g;
+  __shared__ int s_ok;
+  __shared__ float rtab[128];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) s_ticket = static_cast<int>(atomicAdd(a.ctr, 1u));
+  __syncthreads();
+  const int t = s_ticket;
+  const int BH = a.B * a.H;
+  if (t < a.n_work) {
+    // ---- 1. max|x| over part t
+    const int sl = t / a.parts, part = t % a.parts;
+    const int bh = sl % BH, tensor = (sl / BH) & 1, layer = sl / (2 * BH);
+    const int b = bh / a.H, h = bh % a.H;
+    const int t_begin = part * kTicketTokens, t_end = min(a.L, t_begin + kTicketTokens);
+    const uint16_t* x = a.x[layer][tensor] + static_cast<int64_t>(b) * a.L * a.token_stride +
+                        static_cast<int64_t>(h) * kHeadDim + (threadIdx.x & 15) * 8;
+    const int sub = threadIdx.x >> 4;
+    uint4 w[kPasses];
+#pragma unroll
+    for (int u = 0; u < kPasses; ++u) {
+      const int tt = t_begin + u * (kThreads / 16) + sub;
+      w[u] = tt < t_end ? ld_row16(x + static_cast<int64_t>(tt) * a.token_stride) : make_uint4(0, 0, 0, 0);
+    }
+    uint32_t acc = 0;
+#pragma unroll
+    for (int u = 0; u < kPasses; ++u) acc = __vmaxu2(acc, absmax_bits(w[u]));
+    uint32_t m = max(acc & 0xFFFFu, acc >> 16);
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t r = 0;
+#pragma unroll
+      for (int i = 0; i < kWarps; ++i) r = max(r, red[i]);
+      atomicMax(a.ctr + 1 + 2 * sl, r);
+      __threadfence();
+      atomicAdd(a.ctr + 2 + 2 * sl, 1u);
+    }
+  }
+  const int e = t - a.lag;
+  if (e < 0 || e >= a.n_work) return;
+  // ---- 2. encode part e; its rows do not depend on the slice maximum, so they load first
+  const int sl = e / a.parts, part = e % a.parts;
+  const int bh = sl % BH, tensor = (sl / BH) & 1, layer = sl / (2 * BH);
+  const int b = bh / a.H, h = bh % a.H;
+  const int t_begin = part * kTicketTokens, t_end = min(a.L, t_begin + kTicketTokens);
+  const int j = threadIdx.x & 3, tok = threadIdx.x >> 2;  // 4 threads per token, 32 elements each
+  const uint16_t* x = a.x[layer][tensor] + static_cast<int64_t>(b) * a.L * a.token_stride +
+                      static_cast<int64_t>(h) * kHeadDim + j * 32;
+  constexpr int kRowsPerPass = kThreads / 4;
+  constexpr int kEncPass = kTicketTokens / kRowsPerPass;  // 2
+  uint4 w[kEncPass][4];
+#pragma unroll
+  for (int u = 0; u < kEncPass; ++u) {
+    const int tt = t_begin + u * kRowsPerPass + tok;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      w[u][k] = tt < t_end ? ld_row16(x + static_cast<int64_t>(tt) * a.token_stride + 8 * k) : make_uint4(0, 0, 0, 0);
+  }
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const uint32_t* done = a.ctr + 2 + 2 * sl;
+    uint64_t t0 = 0;
+    int it = 0;
+    while (ld_acquire_u32(done) < static_cast<uint32_t>(a.parts)) {
+      const uint64_t now = ptx::globaltimer_ns();
+      if (it++ == 0) t0 = now;
+      if (now - t0 > kWaitLimitNs) {
+        ok = 0;
+        atomicOr(a.status, kStatusTimeout);
+        break;
+      }
+      __nanosleep(64);
+    }
+    const float A = __uint_as_float(ld_acquire_u32(a.ctr + 1 + 2 * sl) << 16);
+    // FP32 scale of this (chunk, head, tensor): g = max|x| / (448 * 6)
+    s_g = (A == 0.0f) ? 0.0f : __fdiv_rn(A, 2688.0f);
+    s_ok = ok;
+    if (ok && part == 0) a.gscale[layer][tensor][static_cast<int64_t>(bh) * a.C + a.slot] = s_g;
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  const Encoder enc = make_encoder(s_g, rtab, threadIdx.x, kThreads);
+  __syncthreads();
+  const int64_t row0 = static_cast<int64_t>(bh) * a.T + static_cast<int64_t>(a.slot) * a.L;
+  uint8_t* codes = a.codes[layer][tensor] + row0 * kCodeBytes + j * 16;
+  uint8_t* scales = a.scales[layer][tensor] + row0 * kScaleBytes + j * 2;
+#pragma unroll
+  for (int u = 0; u < kEncPass; ++u) {
+    const int tt = t_begin + u * kRowsPerPass + tok;
+    if (tt < t_end)
+      encode32_store(w[u], enc, rtab, codes + static_cast<int64_t>(tt) * kCodeBytes,
+                     scales + static_cast<int64_t>(tt) * kScaleBytes);
   }
 }
 
@@ -360,8 +519,8 @@ namespace {
 
 // Cluster size for the single-pass path, or 0 when the chunk does not fit it: about two CTAs
 // per SM over the whole grid, at least 16 tokens and at most kMaxCtaTokens rows per CTA.
-int cluster_size(int units, int L) {
-  int cl = std::max(1, std::min(kMaxCluster, (2 * 148) / std::max(1, units)));
+int cluster_size(int units, int L, int n_sms) {
+  int cl = std::max(1, std::min(kMaxCluster, (2 * n_sms) / std::max(1, units)));
   cl = std::min(cl, std::max(1, L / 16));
   while (cl < kMaxCluster && (L + cl - 1) / cl > kMaxCtaTokens) ++cl;
   return (L + cl - 1) / cl > kMaxCtaTokens ? 0 : cl;
@@ -393,17 +552,21 @@ cudaLaunchConfig_t cluster_config(const nvfp4kv_cache& c, const ClusterPlan& pl,
 // worth taking when every (b, h, tensor) gets its cluster in the first wave (a second wave
 // would wait for the first to finish its whole load-reduce-encode sequence), so the number of
 // co-resident clusters of the shape is asked once per (device, shape).
+PerDeviceOnce g_cluster_attr;
+
 ClusterPlan cluster_plan(const nvfp4kv_cache& c) {
   ClusterPlan pl;
-  const int cl = cluster_size(2 * c.batch * c.heads, c.chunk_tokens);
+  const int sms = current_sm_count();
+  if (sms <= 0) return pl;
+  const int cl = cluster_size(2 * c.batch * c.heads, c.chunk_tokens, sms);
   if (cl == 0 || tensor_map_encoder() == nullptr) return pl;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(quantize_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    kMaxCtaTokens * kHeadDim * 2);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(quantize_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  // function attributes live per device: set them on each device the library runs on
+  const cudaError_t attr_err = g_cluster_attr.run([] {
+    cudaError_t e = cudaFuncSetAttribute(quantize_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kMaxCtaTokens * kHeadDim * 2);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(quantize_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    return e;
   });
   if (attr_err != cudaSuccess) return pl;
   ClusterPlan cand;
@@ -520,6 +683,51 @@ cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, quantize_kernel, a);
+}
+
+size_t quantize_layers_workspace_bytes(int layers, int batch, int heads) {
+  const size_t words = 1 + 2 * static_cast<size_t>(layers) * 2 * batch * heads;
+  return (words * sizeof(uint32_t) + 255) / 256 * 256;
+}
+
+bool quantize_layers_supported(int layers, int batch, int heads, int chunk_tokens) {
+  const int64_t parts = (chunk_tokens + kTicketTokens - 1) / kTicketTokens;
+  const int64_t work = static_cast<int64_t>(layers) * 2 * batch * heads * parts;
+  return layers >= 1 && layers <= kMaxLayers && work + 2 * parts < (int64_t(1) << 31);
+}
+
+cudaError_t launch_quantize_layers(const nvfp4kv_cache* caches, int layers, int slot, const uint16_t* const* k,
+                                   const uint16_t* const* v, int64_t token_stride, void* workspace,
+                                   cudaStream_t stream) {
+  const nvfp4kv_cache& c = caches[0];
+  TicketArgs a;
+  for (int l = 0; l < layers; ++l) {
+    a.x[l][0] = k[l];
+    a.x[l][1] = v[l];
+    a.codes[l][0] = caches[l].k_codes;
+    a.codes[l][1] = caches[l].v_codes;
+    a.scales[l][0] = caches[l].k_scales;
+    a.scales[l][1] = caches[l].v_scales;
+    a.gscale[l][0] = caches[l].k_gscale;
+    a.gscale[l][1] = caches[l].v_gscale;
+  }
+  a.ctr = static_cast<uint32_t*>(workspace);
+  a.status = c.status;
+  a.token_stride = token_stride;
+  a.T = static_cast<int64_t>(c.capacity_chunks) * c.chunk_tokens;
+  a.B = c.batch;
+  a.H = c.heads;
+  a.L = c.chunk_tokens;
+  a.C = c.capacity_chunks;
+  a.slot = slot;
+  a.parts = (c.chunk_tokens + kTicketTokens - 1) / kTicketTokens;
+  a.lag = 2 * a.parts;
+  a.n_work = layers * 2 * c.batch * c.heads * a.parts;
+  // counters start at zero on every call
+  cudaError_t e = cudaMemsetAsync(workspace, 0, quantize_layers_workspace_bytes(layers, c.batch, c.heads), stream);
+  if (e != cudaSuccess) return e;
+  quantize_ticket_kernel<<<a.n_work + a.lag, kThreads, 0, stream>>>(a);
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------------------

@@ -117,3 +117,29 @@ def chunk_kv(w: Workload, slot: int, layer: int = 0) -> tuple[np.ndarray, np.nda
 def queries(w: Workload, layer: int = 0, step: int = 0) -> np.ndarray:
     """bf16 queries of the query chunk (uint16 [B, Lq, H, d]); ``step`` picks a denoising step."""
     return _draw(w, "q", layer, 10_000 + step, w.q_tokens)
+
+
+# ---- the same recipe drawn on the GPU (torch's counter-based generator), for inputs too large to
+# draw on the host in reasonable time (the benchmark's 30-layer rollout).  Not the same bytes as
+# the numpy draws above; the parity tests use those.
+def _device_seed(*key: int) -> int:
+    return int(np.random.SeedSequence(list(key)).generate_state(1, dtype=np.uint64)[0] >> 1)
+
+
+def _device_draw(w: Workload, tensor: str, layer: int, slot: int, tokens: int, device):
+    import torch
+    g = torch.Generator(device=device).manual_seed(_device_seed(w.seed, layer, slot, _TENSOR_ID[tensor], 77))
+    x = torch.randn((w.batch, tokens, w.heads, w.head_dim), generator=g, device=device, dtype=torch.float32)
+    gains = torch.from_numpy(_channel_gains(w, tensor, layer).astype(np.float32)).to(device)
+    return (x * gains).to(torch.bfloat16)
+
+
+def device_chunk_kv(w: Workload, slot: int, layer: int = 0, device="cuda"):
+    """bf16 CUDA tensors K, V [B, Lc, H, d] of chunk ``slot`` of layer ``layer``."""
+    return (_device_draw(w, "k", layer, slot, w.chunk_tokens, device),
+            _device_draw(w, "v", layer, slot, w.chunk_tokens, device))
+
+
+def device_queries(w: Workload, layer: int = 0, step: int = 0, device="cuda"):
+    """bf16 CUDA tensor of the query chunk [B, Lq, H, d]."""
+    return _device_draw(w, "q", layer, 10_000 + step, w.q_tokens, device)

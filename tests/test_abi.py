@@ -86,6 +86,25 @@ def test_attention_slot_list_argument_checks(L):
     assert _attn_slots(L, d, [0, 2, 4, 6, 7], lq=0) == nk.ERR_INVALID_ARG
 
 
+def _attn_ms(L, d, q_chunk=9, sink=1, window=2, start=4, length=2, lq=64):
+    return L.nvfp4_kv_attention_multishot(ctypes.byref(d), 0x80000, lq, 256, q_chunk, sink, window, start,
+                                          length, 0.0, 0x90000, 0, 0xA0000, 1 << 30, None)
+
+
+def test_multishot_argument_checks(L):
+    # paper page, section 4.2: the shot's sink (start, len) is history of the query chunk
+    d = _desc(capacity_chunks=12)
+    assert _attn_ms(L, d, start=-1) == nk.ERR_INVALID_ARG
+    assert _attn_ms(L, d, length=-1) == nk.ERR_INVALID_ARG
+    assert _attn_ms(L, d, start=9, length=2) == nk.ERR_INVALID_ARG   # ends past the query chunk
+    assert _attn_ms(L, d, q_chunk=12) == nk.ERR_INVALID_ARG
+    assert _attn_ms(L, d, window=0) == nk.ERR_INVALID_ARG
+    assert _attn_ms(L, d, sink=-1) == nk.ERR_INVALID_ARG
+    assert _attn_ms(L, d, lq=0) == nk.ERR_INVALID_ARG
+    assert L.nvfp4_kv_attention_multishot(None, 0x80000, 64, 256, 9, 1, 2, 4, 2, 0.0, 0x90000, 0, 0xA0000,
+                                          1 << 30, None) == nk.ERR_INVALID_ARG
+
+
 def test_quantize_argument_checks(L):
     assert L.nvfp4_kv_quantize(None, 0, 0x80000, 0x90000, 256, 0xA0000, 1 << 20, None) == nk.ERR_INVALID_ARG
     assert _quant(L, _desc(head_dim=64)) == nk.ERR_UNSUPPORTED
@@ -135,6 +154,8 @@ def test_valid_arguments_without_a_gpu_report_a_cuda_error(L):
     assert _attn(L, _desc()) == nk.ERR_CUDA
     # four runs, listed out of order and with repeats: valid, so it reaches the device check
     assert _attn_slots(L, _desc(capacity_chunks=12), [9, 0, 4, 5, 0, 7, 9]) == nk.ERR_CUDA
+    assert _attn_ms(L, _desc(capacity_chunks=12)) == nk.ERR_CUDA
+    assert _attn_ms(L, _desc(capacity_chunks=12), start=9, length=1) == nk.ERR_CUDA  # shot = query chunk
     assert L.nvfp4kv_quantize_launches(ctypes.byref(_desc())) == -nk.ERR_CUDA
     assert L.nvfp4kv_debug_wait_timeout(ctypes.byref(_desc()), None) == nk.ERR_CUDA
 

@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 
 import oracle
-from nvfp4_quantised_kv_b200 import KVCache, debug_encode, synthetic
+from nvfp4_quantised_kv_b200 import KVCache, debug_encode, quantize_layers, synthetic
 from tests import special_chunks as sc
 from tests.gpu_util import assert_cache_equal, dev_bf16, make_caches
 
@@ -62,7 +62,7 @@ def test_quantize_matches_oracle_bit_for_bit(key, slots):
 TWO_PASS_TOKENS = 7200
 
 
-@pytest.mark.parametrize("path", ["cluster", "two_pass"])
+@pytest.mark.parametrize("path", ["cluster", "two_pass", "layers"])
 @pytest.mark.parametrize("name", ["fixed0", "fixed-20", "fixed17", "fixed-100", "ties0", "ties-9",
                                   "underflow", "tiny_scale"])
 def test_special_chunks_match_oracle(name, path):
@@ -78,8 +78,12 @@ def test_special_chunks_match_oracle(name, path):
     cache = KVCache(1, 1, L, 2)
     ocache = oracle.Cache(1, 1, 128, L, 2)
     neg = chunk ^ np.uint16(0x8000)  # V gets the negated chunk
-    assert cache.quantize_launches() == (1 if path == "cluster" else 2)
-    cache.quantize(1, dev_bf16(chunk), dev_bf16(neg))
+    if path == "layers":  # the single-launch multi-layer path, as the second of two layers
+        other = KVCache(1, 1, L, 2)
+        quantize_layers([other, cache], 1, [dev_bf16(neg), dev_bf16(chunk)], [dev_bf16(chunk), dev_bf16(neg)])
+    else:
+        assert cache.quantize_launches() == (1 if path == "cluster" else 2)
+        cache.quantize(1, dev_bf16(chunk), dev_bf16(neg))
     ocache.append(1, chunk, neg)
     assert_cache_equal(cache, ocache, [1])
     # the slot not written stays untouched
@@ -130,3 +134,38 @@ def test_quantize_is_deterministic():
     cache.quantize(2, kd, vd)
     for a, b in zip(first, (cache.k_codes, cache.v_scales, cache.k_gscale)):
         assert bool((a == b).all())
+
+
+@pytest.mark.parametrize("batch,heads,chunk_tokens,layers", [(1, 2, 64, 3), (2, 3, 300, 2), (1, 1, 2, 5)])
+def test_quantize_layers_matches_oracle_bit_for_bit(batch, heads, chunk_tokens, layers):
+    # one launch for every layer's new chunk (ragged last parts, many slices, 2-token chunks)
+    w = dataclasses.replace(synthetic.WORKLOADS["tiny"], batch=batch, heads=heads, chunk_tokens=chunk_tokens,
+                            capacity=3)
+    caches = [KVCache(batch, heads, chunk_tokens, 3) for _ in range(layers)]
+    kv = [synthetic.chunk_kv(w, 2, layer) for layer in range(layers)]
+    quantize_layers(caches, 2, [dev_bf16(k) for k, _ in kv], [dev_bf16(v) for _, v in kv])
+    for layer in range(layers):
+        ocache = oracle.Cache(batch, heads, 128, chunk_tokens, 3)
+        ocache.append(2, *kv[layer])
+        assert_cache_equal(caches[layer], ocache, [2])
+        assert int(caches[layer].k_codes[:, :, :2 * chunk_tokens].abs().sum()) == 0  # other slots untouched
+    assert caches[0].read_status() == 0
+
+
+def test_quantize_layers_full_size_equals_per_layer_calls():
+    # four 1.3B-class layers in one launch; layer 0 against the oracle, all against the per-layer call
+    w = synthetic.WORKLOADS["1.3b"]
+    layers = 4
+    caches = [KVCache(w.batch, w.heads, w.chunk_tokens, w.capacity) for _ in range(layers)]
+    refs = [KVCache(w.batch, w.heads, w.chunk_tokens, w.capacity) for _ in range(layers)]
+    kv = [tuple(dev_bf16(x) for x in synthetic.chunk_kv(w, 3, layer)) for layer in range(layers)]
+    ws = quantize_layers(caches, 3, [k for k, _ in kv], [v for _, v in kv])
+    quantize_layers(caches, 3, [k for k, _ in kv], [v for _, v in kv], workspace=ws)  # reused scratch
+    for c, r, (k, v) in zip(caches, refs, kv):
+        r.quantize(3, k, v)
+        for name in ("k_codes", "v_codes", "k_scales", "v_scales", "k_gscale", "v_gscale"):
+            assert bool((getattr(c, name) == getattr(r, name)).all()), name
+    ocache = oracle.Cache(w.batch, w.heads, 128, w.chunk_tokens, w.capacity)
+    ocache.append(3, *synthetic.chunk_kv(w, 3, 0))
+    assert_cache_equal(caches[0], ocache, [3])
+    assert caches[0].read_status() == 0
