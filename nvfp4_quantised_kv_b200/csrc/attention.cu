@@ -22,9 +22,9 @@
 //                             tile (TMA, 128B swizzle) and converts it to fp16 in place
 //   producer warp 8           1-D bulk copies of each KV tile's packed codes + E4M3 scales into
 //                             a ring of shared-memory slots
-//   MMA warp 9                TMEM allocation; tcgen05.mma S = Q K^T (both operands in smem),
+//   MMA warp 12               TMEM allocation; tcgen05.mma S = Q K^T (both operands in smem),
 //                             O += P V (P from TMEM, V from smem), one elected lane
-//   dequant warps 10-15       E2M1 * E4M3 products, exact in fp16, written straight into the
+//   dequant warps 9-11, 13-15 E2M1 * E4M3 products, exact in fp16, written straight into the
 //                             128B-swizzled UMMA operand layout: K (the B operand of Q K^T,
 //                             K-major) and V (the B operand of P V, MN-major)
 // S is computed in sub-tiles of 64 keys, double-buffered in TMEM per query tile (4 x 64 columns
@@ -65,16 +65,22 @@ constexpr int TILE16 = BN * D * 2;                      // one 128 x 128 16-bit 
 constexpr int HALF16 = TILE16 / 2;                      // 128 rows x 64 elements (128 B rows)
 constexpr int MAX_RUNS = kAttnMaxRuns;
 constexpr int kMaxCtas = 1024;
-// Relative cost of one KV tile of a two-tile item and of a one-tile item (the planner's weights).
-constexpr int kWPair = 5, kWSingle = 3;
+// Relative cost of one KV tile of a two-tile item and of a one-tile item (the planner's weights;
+// measured on B200: a one-tile item's KV tile takes about 0.78 of a two-tile item's).
+constexpr int kWPair = 9, kWSingle = 7;
 // Floats of one partial-result slot: O[QT][BM][D], m[QT][BM], l[QT][BM], the reference g_V.
 constexpr int kSlotFloats = QT * BM * D + 2 * QT * BM + 4;
 
 struct Cfg {
   static constexpr int kSoftmaxWarps = 4 * QT;
-  static constexpr int kProducerWarp = kSoftmaxWarps;
-  static constexpr int kMmaWarp = kSoftmaxWarps + 1;
-  static constexpr int kDequantWarp0 = kSoftmaxWarps + 2;
+  // Warps are spread over the SM's four sub-partitions by index mod 4, and every sub-partition
+  // holds two softmax warps.  The two light roles (producer, MMA issue) share sub-partition 0 and
+  // the six dequant warps take two each on sub-partitions 1-3, so no softmax warp shares its
+  // issue slots with the MMA warp.
+  static constexpr int kProducerWarp = kSoftmaxWarps;      // warp 8
+  static constexpr int kMmaWarp = kSoftmaxWarps + 4;       // warp 12
+  // dequant warp index (0..5) of warp w in 9..15 other than the MMA warp
+  __device__ static int dequant_index(int w) { return w < kMmaWarp ? w - kSoftmaxWarps - 1 : w - kSoftmaxWarps - 2; }
   static constexpr int kDequantWarps = 6;  // 2 in the producer/MMA warpgroup + one full warpgroup
   static constexpr int kDequantThreads = 32 * kDequantWarps;
   static_assert(kDequantThreads % 64 == 0, "dequant_tile deals blocks to a multiple of 64 threads");
@@ -330,6 +336,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
   const int cta = blockIdx.x;
   // This CTA's range of (item, KV tile) units; every role walks the same segments.
   const int ubeg = static_cast<int>(plan_cut(p.pl, cta)), uend = static_cast<int>(plan_cut(p.pl, cta + 1));
+  // the merge kernel may be scheduled now; it waits for this whole grid before reading anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int n_dq_warps = C::kDequantWarps;
 
   const uint32_t sbase = ptx::smem_u32(smem);
@@ -795,7 +803,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
       // ========================================================== dequant warps
       // No barrier among the dequant warps: each works through the same tiles on its own, so a
       // warp that gives up after a time-out never leaves the others waiting.
-      const int dt = threadIdx.x - C::kDequantWarp0 * 32;
+      const int dt = C::dequant_index(warp) * 32 + lane;
       float inv_gv = 1.0f;
       int jj = 0;
       bool ok = true;
@@ -863,68 +871,90 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
   }
 }
 
-// Merges the partial results of every work item whose KV tiles were split between CTAs.  Block
-// b - 1 looks at the boundary between CTAs b - 1 and b; the first boundary inside an item merges
-// that item.  One warp per query row: each lane owns 4 of the 128 columns.
+// Merges the partial results of every work item whose KV tiles were split between CTAs.  Blocks
+// (b - 1, rg) look at the boundary between CTAs b - 1 and b; the first boundary inside an item merges
+// that item, rows [16 rg, 16 rg + 16) of its query rows, one warp per row (each lane owns 4 of the
+// 128 columns; lane i loads the running max and sum of part i):
 //   m* = max_k m_k;  O = sum_k O_k 2^(m_k - m*);  l = sum_k l_k 2^(m_k - m*);  out = O g_ref / l
-// (the m_k are whole numbers, so every factor is an exact power of two).
-__global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ AttnParams p) {
+// (the m_k are whole numbers, so every factor is an exact power of two).  Launched as a
+// programmatic dependent of the attention grid: it waits for that grid before reading partials.
+constexpr int kCombineRows = 16;
+
+__global__ void __launch_bounds__(32 * kCombineRows) combine_kernel(const __grid_constant__ AttnParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const Plan& pl = p.pl;
   const int bnd = blockIdx.x + 1;
   const int64_t u = plan_cut(pl, bnd);
   if (u >= pl.units || u % pl.NT == 0) return;
   const int64_t item = u / pl.NT, istart = item * pl.NT, iend = istart + pl.NT;
-  if (plan_cut(pl, bnd - 1) > istart) return;  // an earlier boundary lies inside this item
+  const int bhi = static_cast<int>(item / pl.ipb), k = static_cast<int>(item % pl.ipb);
+  const int m0 = 2 * k * BM, nq = (2 * k + 1 < pl.n_qt) ? 2 : 1;
+  const int r = blockIdx.y * kCombineRows + (threadIdx.x >> 5);  // query row of the item
+  if (blockIdx.y * kCombineRows >= nq * BM || m0 + blockIdx.y * kCombineRows >= p.Lq) return;
   __shared__ int slots[kMaxCtas];
   __shared__ int n_slots;
   if (threadIdx.x == 0) {
     int n = 0;
-    for (int c = bnd - 1; c < pl.G; ++c) {
-      const int64_t cs = plan_cut(pl, c), ce = plan_cut(pl, c + 1);
-      if (cs >= iend) break;
-      if (ce <= istart || cs == ce) continue;
-      slots[n++] = 2 * c + (cs < istart ? 1 : 0);
+    if (plan_cut(pl, bnd - 1) <= istart) {  // otherwise an earlier boundary lies inside this item
+      for (int c = bnd - 1; c < pl.G; ++c) {
+        const int64_t cs = plan_cut(pl, c), ce = plan_cut(pl, c + 1);
+        if (cs >= iend) break;
+        if (ce <= istart || cs == ce) continue;
+        slots[n++] = 2 * c + (cs < istart ? 1 : 0);
+      }
     }
     n_slots = n;
   }
   __syncthreads();
   const int ns = n_slots;
-  const int bhi = static_cast<int>(item / pl.ipb), k = static_cast<int>(item % pl.ipb);
-  const int m0 = 2 * k * BM, nq = (2 * k + 1 < pl.n_qt) ? 2 : 1;
+  const int qrow = m0 + r;
+  if (ns == 0 || r >= nq * BM || qrow >= p.Lq) return;
+  const int lane = threadIdx.x & 31;
   const int b = bhi / p.H, h = bhi % p.H;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float gv = p.part[static_cast<int64_t>(slots[0]) * kSlotFloats + QT * BM * D + 2 * QT * BM];
-  for (int r = warp; r < nq * BM; r += 8) {
-    const int qrow = m0 + r;
-    if (qrow >= p.Lq) continue;
-    float mstar = -INFINITY;
-    for (int i = 0; i < ns; ++i)
-      mstar = fmaxf(mstar, p.part[static_cast<int64_t>(slots[i]) * kSlotFloats + QT * BM * D + r]);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float l = 0.0f;
-    for (int i = 0; i < ns; ++i) {
+  float mstar = -INFINITY;
+  for (int i = lane; i < ns; i += 32)
+    mstar = fmaxf(mstar, p.part[static_cast<int64_t>(slots[i]) * kSlotFloats + QT * BM * D + r]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xFFFFFFFFu, mstar, o));
+  float lsum = 0.0f;
+  for (int i = lane; i < ns; i += 32) {
+    const float* sp = p.part + static_cast<int64_t>(slots[i]) * kSlotFloats;
+    lsum += ptx::ex2(sp[QT * BM * D + r] - mstar) * sp[QT * BM * D + QT * BM + r];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xFFFFFFFFu, lsum, o);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i0 = 0; i0 < ns; i0 += 4) {
+    float4 ov[4];
+    float wv[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {  // four parts' loads in flight
+      const int i = i0 + t < ns ? i0 + t : i0;
       const float* sp = p.part + static_cast<int64_t>(slots[i]) * kSlotFloats;
-      const float wgt = ptx::ex2(sp[QT * BM * D + r] - mstar);
-      const float4 o = reinterpret_cast<const float4*>(sp + r * D)[lane];
-      acc.x += wgt * o.x;
-      acc.y += wgt * o.y;
-      acc.z += wgt * o.z;
-      acc.w += wgt * o.w;
-      l += wgt * sp[QT * BM * D + QT * BM + r];
+      ov[t] = reinterpret_cast<const float4*>(sp + r * D)[lane];
+      wv[t] = i0 + t < ns ? ptx::ex2(sp[QT * BM * D + r] - mstar) : 0.0f;
     }
-    const float inv = gv / l;
-    const int64_t obase = ((static_cast<int64_t>(b) * p.Lq + qrow) * p.H + h) * D + 4 * lane;
-    if (p.out_bf16) {
-      __nv_bfloat162 v0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-      __nv_bfloat162 v1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-      uint2 w;
-      w.x = *reinterpret_cast<uint32_t*>(&v0);
-      w.y = *reinterpret_cast<uint32_t*>(&v1);
-      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + obase) = w;
-    } else {
-      *reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase) =
-          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      acc.x = fmaf(wv[t], ov[t].x, acc.x);
+      acc.y = fmaf(wv[t], ov[t].y, acc.y);
+      acc.z = fmaf(wv[t], ov[t].z, acc.z);
+      acc.w = fmaf(wv[t], ov[t].w, acc.w);
     }
+  }
+  const float gv = p.part[static_cast<int64_t>(slots[0]) * kSlotFloats + QT * BM * D + 2 * QT * BM];
+  const float inv = gv / lsum;
+  const int64_t obase = ((static_cast<int64_t>(b) * p.Lq + qrow) * p.H + h) * D + 4 * lane;
+  if (p.out_bf16) {
+    __nv_bfloat162 v0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    __nv_bfloat162 v1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    uint2 w;
+    w.x = *reinterpret_cast<uint32_t*>(&v0);
+    w.y = *reinterpret_cast<uint32_t*>(&v1);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + obase) = w;
+  } else {
+    *reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   }
 }
 
@@ -1125,8 +1155,16 @@ int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, in
   attention_kernel<<<prm.pl.G, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tm, prm);
   if (cudaGetLastError() != cudaSuccess) return NVFP4KV_ERR_CUDA;
   if (splits) {
-    combine_kernel<<<prm.pl.G - 1, 256, 0, stream>>>(prm);
-    if (cudaGetLastError() != cudaSuccess) return NVFP4KV_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(prm.pl.G - 1, QT * BM / kCombineRows, 1);
+    cfg.blockDim = dim3(32 * kCombineRows, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, combine_kernel, prm) != cudaSuccess) return NVFP4KV_ERR_CUDA;
   }
   return NVFP4KV_OK;
 }

@@ -215,6 +215,34 @@ __device__ __forceinline__ void mma_qk8_w(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+//   QK form with A (Q, fp16 pairs) in TMEM, 8 columns per K = 16 step; B K-major with 128B
+//   swizzle as in mma_qk8_w.
+__device__ __forceinline__ void mma_qk8_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t.reg .b32 blo, bhi, t1, ta;\n\t.reg .b64 db;\n\t"
+      "mov.b64 {blo, bhi}, %2;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.s32 ta, %1, 8;\n\tadd.s32 t1, blo, 2;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 16;\n\tadd.s32 t1, blo, 4;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 24;\n\tadd.s32 t1, blo, 6;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 32;\n\tadd.s32 t1, blo, 1024;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 40;\n\tadd.s32 t1, blo, 1026;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 48;\n\tadd.s32 t1, blo, 1028;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t"
+      "add.s32 ta, %1, 56;\n\tadd.s32 t1, blo, 1030;\n\tmov.b64 db, {t1, bhi};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, 1;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 //   PV form: A (P, fp16) in TMEM, 8 columns per K = 16 step; B MN-major with 128B swizzle,
 //            step k 2048 B further (16 rows of 128 B).
 __device__ __forceinline__ void mma_pv8_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
@@ -339,6 +367,23 @@ __device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[16]
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
+      : "memory");
+}
+
+// 32 lanes x 8 consecutive 32-bit columns, followed by its own wait.
+__device__ __forceinline__ void tmem_ld8_wait(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
       : "memory");
 }
 

@@ -9,7 +9,7 @@ import pytest
 import nvfp4_quantised_kv_b200 as nk
 from tests.test_abi import _desc
 
-W_PAIR, W_SINGLE = 5, 3  # the planner's relative cost of a KV tile of a two-tile / one-tile item
+W_PAIR, W_SINGLE = 9, 7  # the planner's relative cost of a KV tile of a two-tile / one-tile item
 
 
 def _plan(L, d, lq, nt, sms, cta=-1, seg=-1):
