@@ -112,8 +112,8 @@ struct Cfg {
   static constexpr int bKEmpty = bVFull + NST;     // [NST] K stage read by every QK of its tile
   static constexpr int bVEmpty = bKEmpty + NST;    // [NST] V stage read by every PV of its tile
   static constexpr int bTabFull = bVEmpty + NST;   // [NCT] column tables of a tile written
-  static constexpr int bSFull = bTabFull + NCT;    // [QT][2] S sub-tile computed
-  static constexpr int bPFull = bSFull + 2 * QT;   // [QT][2] P sub-tile stored
+  static constexpr int bSFull = bTabFull + NCT;    // [QT] S of a whole KV tile computed
+  static constexpr int bPFull = bSFull + QT;       // [QT][2] P sub-tile stored
   static constexpr int bODone = bPFull + 2 * QT;   // [QT][2] PV of a sub-tile complete
   static constexpr int bDrain = bODone + 2 * QT;
   static constexpr int kNumBars = bDrain + 1;
@@ -349,8 +349,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
     for (int q = 0; q < QT; ++q) {
       ptx::mbar_init(bar(C::bQFull + q), 1);
       ptx::mbar_init(bar(C::bQReady + q), 4);
+      ptx::mbar_init(bar(C::bSFull + q), 1);
       for (int b = 0; b < 2; ++b) {
-        ptx::mbar_init(bar(C::bSFull + 2 * q + b), 1);
         ptx::mbar_init(bar(C::bPFull + 2 * q + b), 4);
         ptx::mbar_init(bar(C::bODone + 2 * q + b), 1);
       }
@@ -475,8 +475,10 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         const int jj = jjb + (hs >> 1);
         const int bf = g & 1, half = hs & 1;
         const uint32_t tS = tS0 + bf * SUB;
-        ok = waitw(bar(C::bSFull + 2 * qt + bf), (g >> 1) & 1, abort_flag, p.status);
-        if (ok && half == 0) ok = waitw(bar(C::bTabFull + jj % NCT), (jj / NCT) & 1, abort_flag, p.status);
+        // S of the whole KV tile arrives with its first sub-tile
+        if (half == 0)
+          ok = waitw(bar(C::bSFull + qt), (g >> 1) & 1, abort_flag, p.status) &&
+               waitw(bar(C::bTabFull + jj % NCT), (jj / NCT) & 1, abort_flag, p.status);
         if (!ok) break;
         ptx::tc_fence_after();
         const int ct = static_cast<int>(jj % NCT);
@@ -725,22 +727,23 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
       // ========================================================== MMA issuer
       // The whole warp runs this loop with warp-uniform values; one elected lane issues each
       // tcgen05 instruction.  kind::f16 instruction descriptors: fp16 x fp16 -> fp32; M = 128.
-      constexpr uint32_t kIdescQK = (1u << 4) |  // A = Q and B = K^ both K-major; N = 64 keys
-                                    (static_cast<uint32_t>(SUB >> 3) << 17) |
+      constexpr uint32_t kIdescQK = (1u << 4) |  // A = Q and B = K^ both K-major; N = 128 keys
+                                    (static_cast<uint32_t>(BN >> 3) << 17) |
                                     (static_cast<uint32_t>(BM >> 4) << 24);
       constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) |  // B = V^ MN-major; N = 128 dims
                                     (static_cast<uint32_t>(D >> 3) << 17) |
                                     (static_cast<uint32_t>(BM >> 4) << 24);
       // Shared-memory descriptors are built once; a step only advances the 14-bit start address
-      // field (address >> 4).  Sub-tile `half` of a K or V stage starts 64 rows (8 KB) in.
+      // field (address >> 4).  Sub-tile `half` of a V stage starts 64 rows (8 KB) in.
       const uint64_t dQ0 = ptx::smem_desc_sw128(sbase + C::oQ, 16, 1024);
       const uint64_t dK0 = ptx::smem_desc_sw128(sbase + C::oK, 16, 1024);
       const uint64_t dV0 = ptx::smem_desc_sw128(sbase + C::oV, HALF16, 1024);
-      auto issue_qk = [&](int q, int bf, int st, int half) {
+      // S = Q K^T of a whole KV tile (N = 128) into both S sub-buffers of query tile q
+      auto issue_qk = [&](int q, int st) {
         const uint64_t dQ = dQ0 + static_cast<uint64_t>((q * TILE16) >> 4);
-        const uint64_t dK = dK0 + static_cast<uint64_t>((st * TILE16 + half * SUB * 128) >> 4);
-        ptx::mma_qk8_w(tmem + (2 * q + bf) * SUB, dQ, dK, kIdescQK, 0u);
-        ptx::mma_commit_w(bar(C::bSFull + 2 * q + bf));
+        const uint64_t dK = dK0 + static_cast<uint64_t>((st * TILE16) >> 4);
+        ptx::mma_qk8_w(tmem + (2 * q) * SUB, dQ, dK, kIdescQK, 0u);
+        ptx::mma_commit_w(bar(C::bSFull + q));
       };
       auto issue_pv = [&](int q, int bf, int st, int half, uint32_t acc) {
         const uint64_t dV = dV0 + static_cast<uint64_t>((st * TILE16 + half * SUB * 128) >> 4);
@@ -758,12 +761,11 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         if (ok) ok = waitw(bar(C::bKFull + st0), static_cast<uint32_t>((jjb / NST) & 1), abort_flag, p.status);
         if (!ok) break;
         ptx::tc_fence_after();
-        // both sub-tiles of the segment's first KV tile, for every query tile
-        for (int q = 0; q < nq; ++q)
-          for (int hs = 0; hs < 2; ++hs) issue_qk(q, (gq[q] + hs) & 1, st0, hs);
+        for (int q = 0; q < nq; ++q) issue_qk(q, st0);  // the segment's first KV tile
         ptx::mma_commit_w(bar(C::bKEmpty + st0));
-        // Per sub-tile hs: PV(q, hs) as soon as softmax q has written P(q, hs), then QK(q, hs + 2)
-        // into the same S buffer; the two query tiles alternate.
+        // Per sub-tile hs: PV(q, hs) as soon as softmax q has written P(q, hs); after the second
+        // sub-tile of a KV tile, QK(q) of the next KV tile into the S buffers those PVs have read
+        // (issue order keeps it behind them).  The two query tiles alternate.
         for (int hs = 0; hs < nh && ok; ++hs) {
           const int jt = jjb + (hs >> 1);
           const int st = static_cast<int>(jt % NST), half = hs & 1;
@@ -775,16 +777,15 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
             ptx::tc_fence_after();
             issue_pv(q, bf, st, half, hs > 0 ? 1u : 0u);
             if (q == nq - 1 && half == 1) ptx::mma_commit_w(bar(C::bVEmpty + st));
-            if (hs + 2 < nh) {
-              const int jt2 = jjb + ((hs + 2) >> 1);
-              const int st2 = static_cast<int>(jt2 % NST);
-              if (q == 0 && half == 0) {
-                ok = waitw(bar(C::bKFull + st2), static_cast<uint32_t>((jt2 / NST) & 1), abort_flag, p.status);
+            if (half == 1 && hs + 1 < nh) {
+              const int st1 = static_cast<int>((jt + 1) % NST);
+              if (q == 0) {
+                ok = waitw(bar(C::bKFull + st1), static_cast<uint32_t>(((jt + 1) / NST) & 1), abort_flag, p.status);
                 if (!ok) break;
                 ptx::tc_fence_after();
               }
-              issue_qk(q, bf, st2, half);
-              if (q == nq - 1 && half == 1) ptx::mma_commit_w(bar(C::bKEmpty + st2));
+              issue_qk(q, st1);
+              if (q == nq - 1) ptx::mma_commit_w(bar(C::bKEmpty + st1));
             }
           }
         }
