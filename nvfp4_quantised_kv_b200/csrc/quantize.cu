@@ -146,24 +146,6 @@ __device__ __forceinline__ void encode_store(uint4 w, const Encoder& e, const fl
   }
 }
 
-// Encodes 32 consecutive elements of one token row (blocks 2j and 2j + 1, four 16-byte words)
-// and stores their 16 code bytes and 2 scale bytes with one 16-byte and one 2-byte store.
-__device__ __forceinline__ void encode32_store(const uint4 (&w)[4], const Encoder& e, const float* rtab,
-                                               uint8_t* code_dst, uint8_t* scale_dst) {
-  uint32_t qc[4], sc[2];
-#pragma unroll
-  for (int blk = 0; blk < 2; ++blk) {
-    uint32_t mb = __vmaxu2(absmax_bits(w[2 * blk]), absmax_bits(w[2 * blk + 1]));
-    mb = max(mb & 0xFFFFu, mb >> 16);
-    sc[blk] = block_scale_code(__uint_as_float(mb << 16), e);
-    const float r = rtab[sc[blk] & 0x7F];
-    qc[2 * blk] = codes8(w[2 * blk], r);
-    qc[2 * blk + 1] = codes8(w[2 * blk + 1], r);
-  }
-  *reinterpret_cast<uint4*>(code_dst) = make_uint4(qc[0], qc[1], qc[2], qc[3]);
-  *reinterpret_cast<uint16_t*>(scale_dst) = static_cast<uint16_t>(sc[0] | (sc[1] << 8));
-}
-
 __global__ void __launch_bounds__(kThreads, 6) amax_kernel(const __grid_constant__ QuantArgs a) {
   const int part = blockIdx.x, bh = blockIdx.y, tensor = blockIdx.z;
   const int b = bh / a.H, h = bh % a.H;
@@ -253,7 +235,8 @@ __global__ void __launch_bounds__(kThreads, 6) quantize_kernel(const __grid_cons
 //   1. reduces max|x| over part t and folds it into its slice's maximum (atomicMax on the bf16
 //      magnitude bits), then counts the part as done;
 //   2. encodes part e = t - lag once every part of e's slice is done, re-reading its rows (still in
-//      L2: at most about lag parts were read since).
+//      L2: lag parts of 32 KB were read since).  The lag exceeds the number of CTAs that can be
+//      resident at once, so that slice is normally complete before the CTA gets there.
 // Step 2 only waits for tickets below t, which belong to CTAs that already started and whose
 // step 1 waits for nothing, so the wait always ends; it is still bounded (the status bit is set
 // if it ever runs out).  The input crosses HBM once for any number of layers.
@@ -273,6 +256,10 @@ struct TicketArgs {
   int n_work;  // slices * parts
 };
 
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -284,7 +271,6 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_ticket_kernel(const __gr
   __shared__ uint32_t red[kWarps];
   __shared__ float s_g;
   __shared__ int s_ok;
-  __shared__ float rtab[128];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) s_ticket = static_cast<int>(atomicAdd(a.ctr, 1u));
   __syncthreads();
@@ -317,8 +303,7 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_ticket_kernel(const __gr
 #pragma unroll
       for (int i = 0; i < kWarps; ++i) r = max(r, red[i]);
       atomicMax(a.ctr + 1 + 2 * sl, r);
-      __threadfence();
-      atomicAdd(a.ctr + 2 + 2 * sl, 1u);
+      red_release_add(a.ctr + 2 + 2 * sl, 1u);  // orders the maximum before the count
     }
   }
   const int e = t - a.lag;
@@ -364,17 +349,39 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_ticket_kernel(const __gr
   }
   __syncthreads();
   if (!s_ok) return;
-  const Encoder enc = make_encoder(s_g, rtab, threadIdx.x, kThreads);
-  __syncthreads();
+  const float g = s_g;
+  Encoder enc;
+  enc.g = g;
+  enc.d = __fmul_rn(6.0f, g);
+  enc.y = g != 0.0f ? __frcp_rn(enc.d) : 0.0f;
+  enc.fast = g != 0.0f && enc.d >= 0x1p-126f && enc.y >= 0x1p-126f && enc.y < 0x1p127f;
   const int64_t row0 = static_cast<int64_t>(bh) * a.T + static_cast<int64_t>(a.slot) * a.L;
   uint8_t* codes = a.codes[layer][tensor] + row0 * kCodeBytes + j * 16;
   uint8_t* scales = a.scales[layer][tensor] + row0 * kScaleBytes + j * 2;
 #pragma unroll
   for (int u = 0; u < kEncPass; ++u) {
     const int tt = t_begin + u * kRowsPerPass + tok;
-    if (tt < t_end)
-      encode32_store(w[u], enc, rtab, codes + static_cast<int64_t>(tt) * kCodeBytes,
-                     scales + static_cast<int64_t>(tt) * kScaleBytes);
+    if (tt >= t_end) continue;
+    uint32_t qc[4], sc[2];
+#pragma unroll
+    for (int blk = 0; blk < 2; ++blk) {
+      uint32_t mb = __vmaxu2(absmax_bits(w[u][2 * blk]), absmax_bits(w[u][2 * blk + 1]));
+      mb = max(mb & 0xFFFFu, mb >> 16);
+      sc[blk] = block_scale_code(__uint_as_float(mb << 16), enc);
+      // r = RN(1 / RN(s * g)); all-zero codes when s is 0 or the reciprocal overflows (the same
+      // operations as the per-code table of make_encoder)
+      const float sv = ptx::e4m3_to_f32(sc[blk]);
+      float r = 0.0f;
+      if (sv != 0.0f) {
+        r = __frcp_rn(__fmul_rn(sv, g));
+        if (r == __int_as_float(0x7F800000)) r = 0.0f;
+      }
+      qc[2 * blk] = codes8(w[u][2 * blk], r);
+      qc[2 * blk + 1] = codes8(w[u][2 * blk + 1], r);
+    }
+    *reinterpret_cast<uint4*>(codes + static_cast<int64_t>(tt) * kCodeBytes) = make_uint4(qc[0], qc[1], qc[2], qc[3]);
+    *reinterpret_cast<uint16_t*>(scales + static_cast<int64_t>(tt) * kScaleBytes) =
+        static_cast<uint16_t>(sc[0] | (sc[1] << 8));
   }
 }
 
@@ -685,6 +692,9 @@ cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k,
   return cudaLaunchKernelEx(&cfg, quantize_kernel, a);
 }
 
+PerDeviceOnce g_ticket_occ;
+int g_ticket_blocks_per_sm = 0;
+
 size_t quantize_layers_workspace_bytes(int layers, int batch, int heads) {
   const size_t words = 1 + 2 * static_cast<size_t>(layers) * 2 * batch * heads;
   return (words * sizeof(uint32_t) + 255) / 256 * 256;
@@ -721,11 +731,18 @@ cudaError_t launch_quantize_layers(const nvfp4kv_cache* caches, int layers, int 
   a.C = c.capacity_chunks;
   a.slot = slot;
   a.parts = (c.chunk_tokens + kTicketTokens - 1) / kTicketTokens;
-  a.lag = 2 * a.parts;
   a.n_work = layers * 2 * c.batch * c.heads * a.parts;
   // counters start at zero on every call
   cudaError_t e = cudaMemsetAsync(workspace, 0, quantize_layers_workspace_bytes(layers, c.batch, c.heads), stream);
   if (e != cudaSuccess) return e;
+  // lag: more tickets than CTAs can be resident (so the slice of e is normally finished when its
+  // encode starts) plus two slices; the re-read rows stay far inside L2
+  e = g_ticket_occ.run([] {
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&g_ticket_blocks_per_sm, quantize_ticket_kernel, kThreads, 0);
+  });
+  const int sms = current_sm_count();
+  if (e != cudaSuccess || g_ticket_blocks_per_sm <= 0 || sms <= 0) return e != cudaSuccess ? e : cudaErrorUnknown;
+  a.lag = g_ticket_blocks_per_sm * sms + 2 * a.parts;
   quantize_ticket_kernel<<<a.n_work + a.lag, kThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
