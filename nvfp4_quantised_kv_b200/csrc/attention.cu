@@ -432,11 +432,13 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
       ok = waitw(bar(C::bQFull + qt), sq & 1, abort_flag, p.status);
       if (!ok) break;
       q_pending = false;
-      // ---- Q row: bf16 -> fp16 in place after a power-of-two prescale 2^-e that keeps the row's
-      // largest |q| below 2^15; row i of S depends on row i of Q only, so each thread scales its
-      // own row and scales its S row back by 2^e with the logit factor.  The conversion is exact
-      // for elements >= 2^(e-14) (fp16's normal range); smaller ones round to fp16's subnormal
-      // spacing 2^(e-24).  No thread waits for another here.
+      // ---- Q row: bf16 -> fp16 in place after a power-of-two prescale 2^-e that brings the row's
+      // largest |q| into [2^14, 2^15) (e = floor(log2 max|q|) - 14, clamped to [-126, 113] so 2^e
+      // and 2^-e are normal floats); row i of S depends on row i of Q only, so each thread scales
+      // its own row and scales its S row back by 2^e with the logit factor.  The conversion is
+      // exact for every element within 2^-28 of the row's largest (fp16's normal range holds
+      // bf16's 8 significant bits); smaller ones round to fp16's subnormal spacing, an absolute
+      // error of at most 2^-39 of the row's largest |q|.  No thread waits for another here.
       float q_unscale = 1.0f, pre_scale = 1.0f;
       uint8_t* qrow = qbase + row * 128;
       {
@@ -448,7 +450,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         }
         mb = max(mb & 0xFFFFu, mb >> 16);
         const int ex = static_cast<int>((mb >> 7) & 0xFF) - 127;  // floor(log2 max|q|)
-        const int e = ex > 14 ? ex - 14 : 0;
+        const int e = min(max(ex - 14, -126), 113);
         q_unscale = __int_as_float((127 + e) << 23);  // 2^e
         pre_scale = __int_as_float((127 - e) << 23);  // 2^-e
       }

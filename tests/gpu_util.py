@@ -70,3 +70,40 @@ def assert_attention_close(got_rows: np.ndarray, want_rows: np.ndarray, what: st
 def gather_rows(out: np.ndarray, rows: np.ndarray) -> np.ndarray:
     """out is [B, Lq, H, d]; rows are (b, h, i) triples."""
     return np.stack([out[b, i, h] for b, h, i in rows])
+
+
+def attention_rows_threaded(qb, ocache, q_chunk, n_sink, window, rows, softmax_scale=0.0,
+                            threads=None):
+    """The oracle's attention of ``rows``, with the rows split over host threads.
+
+    Each thread calls the single-threaded oracle on its own share of the rows (the oracle keeps
+    no state between calls and ctypes releases the interpreter lock), so the result is the same
+    array the one-call form returns, only sooner.
+    """
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    threads = threads or max(1, min(32, os.cpu_count() or 1))
+    parts = [p for p in np.array_split(rows, threads) if len(p)]
+    with ThreadPoolExecutor(len(parts)) as ex:
+        outs = list(ex.map(lambda p: oracle.attention_rows(qb, ocache, q_chunk, n_sink, window, p,
+                                                            softmax_scale), parts))
+    return np.concatenate(outs)
+
+
+def head_rows(w, bh_list) -> np.ndarray:
+    """Every query row (b, h, i) of the listed (b, h) pairs."""
+    return np.array([(b, h, i) for b, h in bh_list for i in range(w.q_tokens)], np.int32)
+
+
+def kv_tiles(chunk_tokens: int, slots) -> int:
+    """128-key tiles of the visible chunks, which are merged into runs of consecutive slots; a
+    tile never crosses a run boundary."""
+    slots = sorted(set(slots))
+    tiles, i = 0, 0
+    while i < len(slots):
+        k = i
+        while k + 1 < len(slots) and slots[k + 1] == slots[k] + 1:
+            k += 1
+        tiles += -(-(k - i + 1) * chunk_tokens // 128)
+        i = k + 1
+    return tiles
