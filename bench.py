@@ -448,18 +448,22 @@ def measure(w, args, dev, rank, world, local, ws, peaks, src, headline):
     return r, rec, clk, steps
 
 
-def traffic_for(key):
-    """DRAM bytes per attention launch from the last ncu capture of this workload, valid only for
-    the attention source they were taken on (null otherwise)."""
+def traffic_for(key, kind="attention"):
+    """DRAM bytes from the last ncu capture of this workload: per attention launch, or per layer of
+    the multi-layer quantiser launch (``kind="quantize"``); valid only for the source file they were
+    taken on (null otherwise)."""
     import hashlib
     prof = os.path.join(ROOT, "profiles", f"traffic_{key}.json")
     if not os.path.exists(prof):
         return None
     with open(prof) as f:
         rec = json.load(f)
-    with open(os.path.join(ROOT, "nvfp4_quantised_kv_b200", "csrc", "attention.cu"), "rb") as f:
+    src = "attention.cu" if kind == "attention" else "quantize.cu"
+    with open(os.path.join(ROOT, "nvfp4_quantised_kv_b200", "csrc", src), "rb") as f:
         src_sha = hashlib.sha256(f.read()).hexdigest()
-    return rec.get("attention_dram_bytes_per_launch") if rec.get("attention_cu_sha256") == src_sha else None
+    if rec.get(f"{kind}_cu_sha256") != src_sha:
+        return None
+    return rec.get("attention_dram_bytes_per_launch" if kind == "attention" else "quantize_dram_bytes_per_layer")
 
 
 def main():
@@ -473,11 +477,18 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="CPU seconds for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub", action="store_true", help="skip the single-layer sub-records")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="layers of a multi-layer workload (default: the workload's own count); a "
+                         "smaller count runs the same per-layer launches on less device memory")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     from nvfp4_quantised_kv_b200 import synthetic
     w = synthetic.WORKLOADS[args.workload]
+    if args.layers and args.layers != w.layers:
+        if w.layers == 1:
+            ap.error("--layers applies to a multi-layer workload")
+        w = synthetic.with_layers(w, args.layers)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -554,7 +565,9 @@ def main():
                          "algorithmic_bytes_per_launch": attn["algorithmic_bytes_per_call"],
                          "algorithmic_hbm_gbs": attn["algorithmic_hbm_gbs"], "launch_us": attn["launch_us"],
                          "ctas": attn["ctas"], "kernels_per_call": attn["kernels_per_call"]},
-            "quantize": {**rec["quantize"], "peak_source": f"{src} HBM copy"},
+            "quantize": {**rec["quantize"], "peak_source": f"{src} HBM copy",
+                         "traffic": (None if traffic_for(w.key, "quantize") is None or rec["quantize"]["layers_per_launch"] == 1
+                                     else traffic_for(w.key, "quantize") * w.layers)},
             "footprint": footprint,
             "e2e": {"value": whole_job_rate(step_flops, world, e2e_ms) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,

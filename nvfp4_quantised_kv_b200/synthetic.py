@@ -13,6 +13,7 @@ so any chunk can be regenerated alone.
 """
 from __future__ import annotations
 
+import dataclasses
 from dataclasses import dataclass
 
 import numpy as np
@@ -107,6 +108,14 @@ def _draw(w: Workload, tensor: str, layer: int, slot: int, tokens: int) -> np.nd
     x = rng.standard_normal((w.batch, tokens, w.heads, w.head_dim))
     x *= _channel_gains(w, tensor, layer)[None, None]
     return f32_to_bf16_bits(x.astype(np.float32))
+
+
+def with_layers(w: Workload, layers: int) -> Workload:
+    """The same workload with ``layers`` layers (each layer's shapes and inputs unchanged)."""
+    if layers < 1:
+        raise ValueError("layers must be positive")
+    name = w.name.replace(f"{w.layers} layers", f"{layers} layer{'s' if layers > 1 else ''}")
+    return dataclasses.replace(w, name=name, layers=layers)
 
 
 def chunk_kv(w: Workload, slot: int, layer: int = 0) -> tuple[np.ndarray, np.ndarray]:
