@@ -23,6 +23,21 @@
  *   E4M3() and E2M1() round to the nearest representable value, ties to the even code,
  *   and clamp to the largest finite magnitude.
  *  Dequantisation [N1]: x_hat = E2M1(q) * E4M3(s) * g, evaluated in fp64 (exact).
+ *
+ *  The pages' own recipe for the cache [N2]: "K-smoothing" of K and "adaptive scale selection"
+ *  of V within each chunk, with the candidate scale targets {4, 6} [N3], [P1 sec. A.2].  The
+ *  pages name both and define neither; the readings taken here:
+ *   K-smoothing: mu_i = (float)((sum over t of x[t][i], in fp64, t = 0, 1, ... in order) / L),
+ *     the channel mean of the chunk's keys of one head; the chunk is quantised as above from
+ *     x'[t][i] = x[t][i] - mu_i (one fp32 subtraction), and the key the cache stands for is
+ *     x_hat' + mu (mu stored in fp32 beside the chunk).
+ *   Adaptive scale (target T in {6, 4}): for every block both targets are tried,
+ *       s_T = E4M3(a_b / (T * g)),  q_i = E2M1(x_i * 1 / (decode(s_T) * g)),
+ *     and the one with the smaller squared error E_T = sum over the block's 16 elements, in
+ *     order, of (x_i - E2M1(q_i) * E4M3(s_T) * g)^2 (fp64, each product, difference, square
+ *     and sum rounded once) is kept; ties keep 6.  g is unchanged (A / (448 * 6)), so a block
+ *     near the chunk maximum whose target-4 scale would exceed 448 saturates, and keeps 6 unless
+ *     the saturated candidate is strictly better.
  *  Attention [P1' sec. 4.2], [P1'' sec. 2.1]: a query row of chunk t attends to the keys of
  *   the visible chunks V(t) = {c < n_sink} U {t - window < c <= t} (duplicates removed), in
  *   fp64: s_j = sigma * q . k_hat_j, p_j = exp(s_j - max_j s_j), o = sum p_j v_hat_j / sum p_j.
@@ -121,10 +136,28 @@ void oracle_e4m3_encode_array(const float* x, int64_t n, uint8_t* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_encode(x[i]);
 }
 
-int oracle_quantize_chunk(const uint16_t* x, int32_t B, int32_t L, int32_t H, int32_t d,
-                          int64_t token_stride, uint8_t* codes, uint8_t* scales, float* gscale) {
+int oracle_key_mean(const uint16_t* x, int32_t B, int32_t L, int32_t H, int32_t d,
+                    int64_t token_stride, float* mean) {
+  if (!x || !mean || B <= 0 || L <= 0 || H <= 0 || d <= 0 || token_stride < static_cast<int64_t>(H) * d)
+    return -1;
+  IeeeMode ieee;
+  for (int32_t b = 0; b < B; ++b)
+    for (int32_t h = 0; h < H; ++h)
+      for (int32_t i = 0; i < d; ++i) {
+        double sum = 0.0;
+        for (int32_t t = 0; t < L; ++t)  /* token order */
+          sum += static_cast<double>(bf16_bits_to_float(
+              x[(static_cast<int64_t>(b) * L + t) * token_stride + static_cast<int64_t>(h) * d + i]));
+        mean[(static_cast<int64_t>(b) * H + h) * d + i] = static_cast<float>(sum / L);
+      }
+  return 0;
+}
+
+int oracle_quantize_chunk_ex(const uint16_t* x, int32_t B, int32_t L, int32_t H, int32_t d,
+                             int64_t token_stride, const float* mean, int32_t adaptive_scale,
+                             uint8_t* codes, uint8_t* scales, float* gscale) {
   if (!x || !codes || !scales || !gscale || B <= 0 || L <= 0 || H <= 0 || d <= 0 || d % 16 != 0 ||
-      token_stride < static_cast<int64_t>(H) * d)
+      token_stride < static_cast<int64_t>(H) * d || (adaptive_scale != 0 && adaptive_scale != 1))
     return -1;
   IeeeMode ieee;
   const int nblk = d / 16;
@@ -132,9 +165,11 @@ int oracle_quantize_chunk(const uint16_t* x, int32_t B, int32_t L, int32_t H, in
   const float kFp4Max = 6.0f;    /* M_FP4 */
   for (int32_t b = 0; b < B; ++b) {
     for (int32_t h = 0; h < H; ++h) {
+      /* the element to quantise: the bf16 input, less the channel mean when K is smoothed */
       auto elem = [&](int32_t t, int32_t i) {
-        return bf16_bits_to_float(x[(static_cast<int64_t>(b) * L + t) * token_stride +
-                                    static_cast<int64_t>(h) * d + i]);
+        const float v = bf16_bits_to_float(x[(static_cast<int64_t>(b) * L + t) * token_stride +
+                                             static_cast<int64_t>(h) * d + i]);
+        return mean ? v - mean[(static_cast<int64_t>(b) * H + h) * d + i] : v;
       };
       /* FP32 scale of this (chunk, head). */
       float A = 0.0f;
@@ -151,29 +186,54 @@ int oracle_quantize_chunk(const uint16_t* x, int32_t B, int32_t L, int32_t H, in
         for (int blk = 0; blk < nblk; ++blk) {
           float ab = 0.0f;
           for (int k = 0; k < 16; ++k) ab = std::fmax(ab, std::fabs(elem(t, blk * 16 + k)));
-          uint8_t s_code = 0;
-          if (ab != 0.0f && g != 0.0f) {
-            const float denom = kFp4Max * g;
-            const float s_raw = ab / denom;
-            s_code = oracle_e4m3_encode(s_raw);
+          /* one candidate per scale target: target 6, and target 4 when the scale is adaptive */
+          uint8_t best_s = 0, best_q[16] = {0};
+          double best_err = 0.0;
+          const int n_targets = adaptive_scale ? 2 : 1;
+          for (int cand = 0; cand < n_targets; ++cand) {
+            const float target = cand == 0 ? kFp4Max : 4.0f;
+            uint8_t s_code = 0, q[16] = {0};
+            if (ab != 0.0f && g != 0.0f) {
+              const float denom = target * g;
+              const float s_raw = ab / denom;
+              s_code = oracle_e4m3_encode(s_raw);
+            }
+            const float s = static_cast<float>(oracle_e4m3_decode(s_code));
+            if (s != 0.0f) {
+              const float sg = s * g;
+              const float r = 1.0f / sg;
+              if (std::isfinite(r)) /* else the scale product underflowed: codes stay 0 */
+                for (int k = 0; k < 16; ++k) q[k] = oracle_e2m1_encode(elem(t, blk * 16 + k) * r);
+            }
+            double err = 0.0;
+            if (adaptive_scale)
+              for (int k = 0; k < 16; ++k) {
+                const double xhat = oracle_e2m1_decode(q[k]) * oracle_e4m3_decode(s_code) * static_cast<double>(g);
+                const double diff = static_cast<double>(elem(t, blk * 16 + k)) - xhat;
+                const double sq = diff * diff;
+                err = err + sq;
+              }
+            if (cand == 0 || err < best_err) { /* strictly smaller: ties keep target 6 */
+              best_err = err;
+              best_s = s_code;
+              for (int k = 0; k < 16; ++k) best_q[k] = q[k];
+            }
           }
-          srow[blk] = s_code;
-          const float s = static_cast<float>(oracle_e4m3_decode(s_code));
-          if (s == 0.0f) continue; /* codes stay 0 */
-          const float sg = s * g;
-          const float r = 1.0f / sg;
-          if (!std::isfinite(r)) continue; /* scale product underflowed: codes stay 0 */
+          srow[blk] = best_s;
           for (int k = 0; k < 16; ++k) {
             const int i = blk * 16 + k;
-            const float y = elem(t, i) * r;
-            const uint8_t q = oracle_e2m1_encode(y);
-            crow[i / 2] |= static_cast<uint8_t>((i % 2 == 0) ? q : (q << 4));
+            crow[i / 2] |= static_cast<uint8_t>((i % 2 == 0) ? best_q[k] : (best_q[k] << 4));
           }
         }
       }
     }
   }
   return 0;
+}
+
+int oracle_quantize_chunk(const uint16_t* x, int32_t B, int32_t L, int32_t H, int32_t d,
+                          int64_t token_stride, uint8_t* codes, uint8_t* scales, float* gscale) {
+  return oracle_quantize_chunk_ex(x, B, L, H, d, token_stride, nullptr, 0, codes, scales, gscale);
 }
 
 int oracle_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gscale, int32_t B,
@@ -237,7 +297,8 @@ int attention_over_slots(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, in
                          const uint8_t* k_codes, const uint8_t* k_scales, const float* k_gscale,
                          const uint8_t* v_codes, const uint8_t* v_scales, const float* v_gscale,
                          int32_t chunk_tokens, int32_t capacity, const int32_t* vis, int nvis,
-                         double softmax_scale, const int32_t* rows, int32_t n_rows, double* out) {
+                         double softmax_scale, const int32_t* rows, int32_t n_rows, double* out,
+                         const float* k_mean) {
   if (!q || !k_codes || !k_scales || !k_gscale || !v_codes || !v_scales || !v_gscale || !rows ||
       !out || B <= 0 || Lq <= 0 || H <= 0 || d <= 0 || d % 16 != 0 || chunk_tokens <= 0 ||
       capacity <= 0 || n_rows < 0 || q_token_stride < static_cast<int64_t>(H) * d || nvis < 0)
@@ -255,6 +316,12 @@ int attention_over_slots(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, in
       const uint8_t c = (i % 2 == 0) ? (byte & 0xF) : (byte >> 4);
       dst[i] = oracle_e2m1_decode(c) * oracle_e4m3_decode(scales[row * (d / 16) + i / 16]) * g;
     }
+  };
+  /* a smoothed key is x_hat' + mu of its chunk (mu: [B][H][capacity][d] fp32) */
+  auto add_mean = [&](int32_t b, int32_t h, int64_t t, double* dst) {
+    if (!k_mean) return;
+    const float* mu = k_mean + ((static_cast<int64_t>(b) * H + h) * capacity + t / chunk_tokens) * d;
+    for (int32_t i = 0; i < d; ++i) dst[i] += static_cast<double>(mu[i]);
   };
 
   /* The visible keys of one (b, h), dequantised once and reused for every requested row of
@@ -274,6 +341,7 @@ int attention_over_slots(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, in
     if (b != cached_b || h != cached_h) {
       for (size_t k = 0; k < nk; ++k) {
         dequant_row(k_codes, k_scales, k_gscale, b, h, keys[k], &khat[k * d]);
+        add_mean(b, h, keys[k], &khat[k * d]);
         dequant_row(v_codes, v_scales, v_gscale, b, h, keys[k], &vhat[k * d]);
       }
       cached_b = b;
@@ -320,16 +388,17 @@ int oracle_attention_rows(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, i
   if (nvis < 0) return -1;
   return attention_over_slots(q, B, Lq, H, d, q_token_stride, k_codes, k_scales, k_gscale, v_codes,
                               v_scales, v_gscale, chunk_tokens, capacity, vis.data(), nvis,
-                              softmax_scale, rows, n_rows, out);
+                              softmax_scale, rows, n_rows, out, nullptr);
 }
 
-int oracle_attention_rows_slots(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, int32_t d,
-                                int64_t q_token_stride,
-                                const uint8_t* k_codes, const uint8_t* k_scales, const float* k_gscale,
-                                const uint8_t* v_codes, const uint8_t* v_scales, const float* v_gscale,
-                                int32_t chunk_tokens, int32_t capacity, const int32_t* slots,
-                                int32_t n_slots, double softmax_scale, const int32_t* rows,
-                                int32_t n_rows, double* out) {
+int oracle_attention_rows_slots_kmean(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, int32_t d,
+                                      int64_t q_token_stride,
+                                      const uint8_t* k_codes, const uint8_t* k_scales, const float* k_gscale,
+                                      const float* k_mean,
+                                      const uint8_t* v_codes, const uint8_t* v_scales, const float* v_gscale,
+                                      int32_t chunk_tokens, int32_t capacity, const int32_t* slots,
+                                      int32_t n_slots, double softmax_scale, const int32_t* rows,
+                                      int32_t n_rows, double* out) {
   if (capacity <= 0 || !slots || n_slots < 1) return -1;
   std::vector<char> listed(static_cast<size_t>(capacity), 0);  /* the union of the listed slots */
   for (int32_t i = 0; i < n_slots; ++i) {
@@ -341,7 +410,19 @@ int oracle_attention_rows_slots(const uint16_t* q, int32_t B, int32_t Lq, int32_
     if (listed[static_cast<size_t>(c)]) vis.push_back(c);
   return attention_over_slots(q, B, Lq, H, d, q_token_stride, k_codes, k_scales, k_gscale, v_codes,
                               v_scales, v_gscale, chunk_tokens, capacity, vis.data(),
-                              static_cast<int>(vis.size()), softmax_scale, rows, n_rows, out);
+                              static_cast<int>(vis.size()), softmax_scale, rows, n_rows, out, k_mean);
+}
+
+int oracle_attention_rows_slots(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, int32_t d,
+                                int64_t q_token_stride,
+                                const uint8_t* k_codes, const uint8_t* k_scales, const float* k_gscale,
+                                const uint8_t* v_codes, const uint8_t* v_scales, const float* v_gscale,
+                                int32_t chunk_tokens, int32_t capacity, const int32_t* slots,
+                                int32_t n_slots, double softmax_scale, const int32_t* rows,
+                                int32_t n_rows, double* out) {
+  return oracle_attention_rows_slots_kmean(q, B, Lq, H, d, q_token_stride, k_codes, k_scales, k_gscale,
+                                           nullptr, v_codes, v_scales, v_gscale, chunk_tokens, capacity,
+                                           slots, n_slots, softmax_scale, rows, n_rows, out);
 }
 
 }  // extern "C"

@@ -21,7 +21,12 @@
  *         elements (1 sign, 2 exponent, 1 mantissa bit), an E4M3 scale per 16 elements,
  *         an FP32 scale on top; dequantisation is the product of the three.
  *   [N2]  reading note, "The inference infrastructure": the KV cache is re-quantised at
- *         frame-chunk granularity; storage goes from 4*Tc*H*d to 9/8*Tc*H*d bytes.
+ *         frame-chunk granularity; storage goes from 4*Tc*H*d to 9/8*Tc*H*d bytes; within a
+ *         chunk, K-smoothing is applied to K and adaptive scale selection to V.
+ *   [N3]  reading note, "Engineering details of NVFP4 training" (few-step distillation): the
+ *         adaptive scale search draws its candidate scale magnitudes from {4, 6}; paper page,
+ *         section A.2, names adaptive block-scale selection ("Four Over Six", its reference [12])
+ *         as a way to lower NVFP4 quantisation error.
  *
  * Cache format the oracle reads and writes (one tensor, K or V):
  *   codes  uint8 [B][H][T][d/2]   element 2j in the low nibble of byte j, 2j+1 in the high
@@ -54,6 +59,20 @@ void oracle_e4m3_encode_array(const float* x, int64_t n, uint8_t* out);
  * Returns 0, or -1 for bad sizes (d not a multiple of 16, non-positive sizes). */
 int oracle_quantize_chunk(const uint16_t* x, int32_t B, int32_t L, int32_t H, int32_t d,
                           int64_t token_stride, uint8_t* codes, uint8_t* scales, float* gscale);
+
+/* K-smoothing [N2]: the channel mean of one chunk's keys per (b, h), as the fp32 rounding of the
+ * fp64 sum over the chunk's tokens in token order divided by L.  mean: [B][H][d].  Returns 0 / -1. */
+int oracle_key_mean(const uint16_t* x, int32_t B, int32_t L, int32_t H, int32_t d,
+                    int64_t token_stride, float* mean);
+
+/* oracle_quantize_chunk with the pages' two recipe options [N2], [N3]:
+ *   mean           : NULL, or [B][H][d]: quantise x - mean (one fp32 subtraction per element)
+ *   adaptive_scale : 0, or 1 to choose each block's scale target from {6, 4} by the smaller fp64
+ *                    squared error (ties keep 6); g stays A / (448 * 6).
+ * With mean NULL and adaptive_scale 0 it is oracle_quantize_chunk.  Returns 0 or -1. */
+int oracle_quantize_chunk_ex(const uint16_t* x, int32_t B, int32_t L, int32_t H, int32_t d,
+                             int64_t token_stride, const float* mean, int32_t adaptive_scale,
+                             uint8_t* codes, uint8_t* scales, float* gscale);
 
 /* Dequantise tokens of a cache tensor into fp64: out[B][H][T][d] = e2m1 * e4m3 * gscale. */
 int oracle_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gscale,
@@ -97,6 +116,17 @@ int oracle_attention_rows_slots(const uint16_t* q, int32_t B, int32_t Lq, int32_
                                 int32_t chunk_tokens, int32_t capacity, const int32_t* slots,
                                 int32_t n_slots, double softmax_scale, const int32_t* rows,
                                 int32_t n_rows, double* out);
+
+/* oracle_attention_rows_slots over smoothed keys: key t of chunk c of (b, h) is x_hat' + mu with
+ * mu = k_mean[((b*H + h)*capacity + c)*d ...] (fp32); k_mean NULL gives oracle_attention_rows_slots. */
+int oracle_attention_rows_slots_kmean(const uint16_t* q, int32_t B, int32_t Lq, int32_t H, int32_t d,
+                                      int64_t q_token_stride,
+                                      const uint8_t* k_codes, const uint8_t* k_scales, const float* k_gscale,
+                                      const float* k_mean,
+                                      const uint8_t* v_codes, const uint8_t* v_scales, const float* v_gscale,
+                                      int32_t chunk_tokens, int32_t capacity, const int32_t* slots,
+                                      int32_t n_slots, double softmax_scale, const int32_t* rows,
+                                      int32_t n_rows, double* out);
 
 #ifdef __cplusplus
 }
