@@ -223,7 +223,7 @@ def config_of(w):
 class Runner:
     """Caches, inputs and outputs of one workload on one GPU, and its timed step."""
 
-    def __init__(self, w, dev, rank, ws):
+    def __init__(self, w, dev, rank, ws, recipe=False):
         import torch
         import nvfp4_quantised_kv_b200 as nk
         from nvfp4_quantised_kv_b200 import synthetic
@@ -237,7 +237,7 @@ class Runner:
             layers = []
             for layer in range(w.layers):
                 cache = nk.KVCache(w.batch, w.heads, w.chunk_tokens, w.capacity, q_tokens_max=w.q_tokens,
-                                   device=dev, workspace=ws)
+                                   device=dev, workspace=ws, smooth_k=recipe, adaptive_v=recipe)
                 for slot in hist:
                     k, v = synthetic.device_chunk_kv(ws_w, slot, layer, dev)
                     cache.quantize(slot, k, v)
@@ -247,7 +247,7 @@ class Runner:
                 layers.append(dict(cache=cache, k=k, v=v, q=q, out=out))
             self.sets.append(layers)
         # the multi-layer step quantises all layers' new chunks with one launch
-        self.batched = w.layers > 1
+        self.batched = w.layers > 1 and not recipe
         self.qws = None
         if self.batched:
             S = self.sets[0]
@@ -410,9 +410,9 @@ def attention_kernels_per_call(w):
     return out[1], out[0]
 
 
-def measure(w, args, dev, rank, world, local, ws, peaks, src, headline):
+def measure(w, args, dev, rank, world, local, ws, peaks, src, headline, recipe=False):
     import nvfp4_quantised_kv_b200 as nk  # noqa: F401
-    r = Runner(w, dev, rank, ws)
+    r = Runner(w, dev, rank, ws, recipe)
     steps = args.steps if headline else max(5, args.steps // 2)
     ms, t_quant, t_attn, clk = r.timed(steps, args.warmup, world, headline and rank == 0, local)
     ms, t_quant, t_attn = max_over_ranks([ms, t_quant, t_attn], dev)
@@ -435,6 +435,7 @@ def measure(w, args, dev, rank, world, local, ws, peaks, src, headline):
                      "layers_per_launch": w.layers if r.batched else 1,
                      "kernels": ("quantize_ticket_kernel (one launch for all layers, after a counter memset)"
                                  if r.batched else
+                                 "key_mean_kernel + recipe_amax_kernel + recipe_encode_kernel" if recipe else
                                  "quantize_cluster_kernel" if q_launches == 1 else "amax_kernel + quantize_kernel"),
                      "algorithmic_bytes_per_step": w.layers * quant_bytes},
         "gpu_launches_per_step": (q_launches if r.batched else w.layers * q_launches) + w.layers * w.attn_calls * a_kernels,
@@ -544,6 +545,13 @@ def main():
             subs[key] = rec2
             del r2
             torch.cuda.empty_cache()
+        # the pages' recipe options (K-smoothing of K, adaptive {4, 6} scales of V) on the 1.3B layer
+        r2, rec2, _, _ = measure(synthetic.WORKLOADS["1.3b"], args, dev, rank, world, local, ws, peaks, src,
+                                 headline=False, recipe=True)
+        rec2["options"] = "K_SMOOTH | V_ADAPTIVE_SCALE"
+        subs["1.3b+recipe"] = rec2
+        del r2
+        torch.cuda.empty_cache()
 
     if rank == 0:
         attn = rec["attention"]

@@ -26,6 +26,22 @@
  *      r   = 1 / (s_b * g);  q_i = E2M1_rn_satfinite(x_i * r) (all 0 if s_b == 0 or r is inf)
  * Dequantisation: x_hat = E2M1(q) * E4M3(s) * g.
  *
+ * Recipe options (nvfp4kv_cache.flags).  The reading note, "The inference infrastructure", applies
+ * "K-smoothing" to K and "adaptive scale selection" to V within each chunk, and "Engineering
+ * details of NVFP4 training" draws the candidate scale magnitudes from {4, 6}; the paper page,
+ * section A.2, cites adaptive block-scale selection ("Four Over Six") for lower NVFP4 error.  The
+ * pages define neither; this library reads them as:
+ *  NVFP4KV_K_SMOOTH: per (chunk, head) the channel mean of the chunk's keys,
+ *      mu_e = fp32( (sum over t = 0, 1, ... of x[t][e], in fp64 in token order) / chunk_tokens ),
+ *    is stored in k_mean and the chunk is quantised as above from x' = x - mu (one fp32
+ *    subtraction per element); the key the cache holds is x_hat' + mu, and attention adds the
+ *    per-(query row, chunk) term q . mu to every logit of the chunk's keys.
+ *  NVFP4KV_V_ADAPTIVE_SCALE: per block of V both scale targets T = 6 and T = 4 are tried
+ *    (s_b = E4M3(max_b|x| / (T * g)), codes as above); the one with the smaller squared error
+ *    sum over the block's 16 elements, in order, of (x_i - E2M1(q_i) * E4M3(s_b) * g)^2 (fp64,
+ *    each operation rounded once) is kept, ties keep 6.  g is unchanged; dequantisation and
+ *    attention read such blocks as any other.
+ *
  * CONVENTIONS (all entry points)
  *  - Every pointer named "device" is CUDA device memory owned by the caller; the library
  *    never allocates or frees device memory.  It keeps no state between calls other than
@@ -66,7 +82,10 @@ typedef enum { NVFP4KV_OUT_F32 = 0, NVFP4KV_OUT_BF16 = 1 } nvfp4kv_out_dtype;
  *   k_scales, v_scales uint8 [batch][heads][T][head_dim/16]  E4M3 block scales
  *   k_gscale, v_gscale fp32  [batch][heads][capacity_chunks] FP32 scale per chunk
  *   status             uint32, one word; zero it once before first use
- * Every array must start on a 16-byte boundary. */
+ *   k_mean             fp32  [batch][heads][capacity_chunks][head_dim] (NVFP4KV_K_SMOOTH only)
+ * Every array must start on a 16-byte boundary.  flags with bits other than the two options,
+ * or NVFP4KV_K_SMOOTH without k_mean, is NVFP4KV_ERR_INVALID_ARG for every call; one cache keeps
+ * its flags for its whole life (its slots are read as they were written). */
 typedef struct {
   int32_t batch;
   int32_t heads;
@@ -80,7 +99,13 @@ typedef struct {
   float* k_gscale;
   float* v_gscale;
   uint32_t* status;
+  uint32_t flags;  /* 0, or recipe options: NVFP4KV_K_SMOOTH | NVFP4KV_V_ADAPTIVE_SCALE */
+  float* k_mean;   /* with NVFP4KV_K_SMOOTH: fp32 [batch][heads][capacity_chunks][head_dim], the
+                      channel mean of each chunk slot's keys; else unused (may be NULL) */
 } nvfp4kv_cache;
+
+/* Recipe option bits of nvfp4kv_cache.flags (see the file header). */
+enum { NVFP4KV_K_SMOOTH = 1u, NVFP4KV_V_ADAPTIVE_SCALE = 2u };
 
 /* Bytes of each cache array for the given shape (per tensor, K or V): codes, scales and
  * FP32 scales.  Any output pointer may be NULL.  Returns NVFP4KV_OK or
@@ -106,9 +131,11 @@ size_t nvfp4kv_workspace_bytes(const nvfp4kv_cache* cache, int32_t q_tokens);
  *                   multiple of 8
  *   workspace       device scratch of at least nvfp4kv_workspace_bytes() bytes, 16-byte
  *                   aligned; its contents on entry do not matter
- * Writes codes, scales and the FP32 scales of slot `chunk_slot` for every (b, h); nothing
- * else in the cache is touched.  Bit-for-bit deterministic, and the same bits whichever of the
- * two kernel paths runs (nvfp4kv_quantize_launches tells which).
+ * Writes codes, scales and the FP32 scales of slot `chunk_slot` for every (b, h) (and, with
+ * NVFP4KV_K_SMOOTH, the slot's channel means in k_mean); nothing else in the cache is touched.
+ * Bit-for-bit deterministic, and the same bits whichever kernel path runs
+ * (nvfp4kv_quantize_launches tells which; a cache with recipe options always takes the
+ * two-pass path, after a channel-mean kernel when K is smoothed).
  * Errors: NVFP4KV_ERR_INVALID_ARG (null, misaligned, slot out of range, bad stride),
  * NVFP4KV_ERR_UNSUPPORTED, NVFP4KV_ERR_WORKSPACE, NVFP4KV_ERR_CUDA (launch failed); a device
  * wait that ran out sets the status bit of NVFP4KV_ERR_DEVICE_TIMEOUT. */
@@ -131,7 +158,8 @@ int nvfp4_kv_quantize(const nvfp4kv_cache* cache, int32_t chunk_slot, const void
  *                  contents on entry do not matter
  * A device wait that runs out sets the timeout bit in caches[0]'s status word.  Errors as for
  * nvfp4_kv_quantize; NVFP4KV_ERR_INVALID_ARG also for caches of different shapes and
- * NVFP4KV_ERR_UNSUPPORTED for more than 64 layers or more than 2^31 parts. */
+ * NVFP4KV_ERR_UNSUPPORTED for more than 64 layers, more than 2^31 parts, or caches with recipe
+ * options (quantise those one layer at a time with nvfp4_kv_quantize). */
 int nvfp4_kv_quantize_layers(const nvfp4kv_cache* caches, int32_t n_layers, int32_t chunk_slot,
                              const void* const* k_bf16, const void* const* v_bf16, int64_t token_stride,
                              void* workspace, size_t workspace_bytes, void* cuda_stream);
@@ -175,9 +203,13 @@ int nvfp4_kv_quantize_static_scratch(const nvfp4kv_cache* cache, int32_t chunk_s
  *   softmax_scale <= 0 selects 1/sqrt(head_dim)
  *   workspace  device scratch of at least nvfp4kv_workspace_bytes(cache, q_tokens) bytes (with
  *              the same device current); contents on entry do not matter
+ * With NVFP4KV_K_SMOOTH, k_hat_j is x_hat'_j + mu(chunk of j): the kernel adds scale * q_i . mu
+ * per (query row, chunk) to the logits; such caches need chunk_tokens >= 128 (else
+ * NVFP4KV_ERR_UNSUPPORTED), so that a 128-key tile spans at most two chunks.
  * One launch of a persistent kernel (one CTA per SM), followed by a small merge kernel when some
- * work item's KV tiles were split between CTAs.  Chunk slots outside V are never read.  Errors as for nvfp4_kv_quantize; window_chunks < 1,
- * n_sink_chunks < 0 or q_chunk outside [0, capacity) give NVFP4KV_ERR_INVALID_ARG. */
+ * work item's KV tiles were split between CTAs.  Chunk slots outside V are never read.  Errors as
+ * for nvfp4_kv_quantize; window_chunks < 1, n_sink_chunks < 0 or q_chunk outside
+ * [0, capacity) give NVFP4KV_ERR_INVALID_ARG. */
 int nvfp4_kv_attention(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q_tokens,
                        int64_t q_token_stride, int32_t q_chunk, int32_t n_sink_chunks,
                        int32_t window_chunks, float softmax_scale, void* out, int32_t out_dtype,
@@ -217,7 +249,8 @@ int nvfp4_kv_attention_multishot(const nvfp4kv_cache* cache, const void* q_bf16,
 /* Dequantise chunk slots [first_slot, first_slot + n_slots) of K (which == 0) or V
  * (which == 1) into device fp32 out[batch][heads][n_slots*chunk_tokens][head_dim]: the
  * pages' dequantisation step on its own, for tests and diagnostics.  Each value is the
- * exact E2M1 * E4M3 product times the FP32 scale, rounded once to fp32. */
+ * exact E2M1 * E4M3 product times the FP32 scale, rounded once to fp32; for K of a cache with
+ * NVFP4KV_K_SMOOTH the chunk's channel mean is then added (a second fp32 rounding). */
 int nvfp4_kv_dequantize(const nvfp4kv_cache* cache, int32_t which, int32_t first_slot,
                         int32_t n_slots, float* out, void* cuda_stream);
 

@@ -26,6 +26,8 @@ ERR_WORKSPACE = 5
 OUT_F32 = 0
 OUT_BF16 = 1
 HEAD_DIM = 128
+K_SMOOTH = 1  # recipe option: K-smoothing of K (channel mean per chunk, added back in attention)
+V_ADAPTIVE_SCALE = 2  # recipe option: per-block scale target chosen from {6, 4} for V
 
 # Every function the C header declares, with its ctypes signature.
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -36,7 +38,7 @@ class CacheDesc(ctypes.Structure):
     _fields_ = [("batch", _i32), ("heads", _i32), ("head_dim", _i32), ("chunk_tokens", _i32),
                 ("capacity_chunks", _i32), ("k_codes", _vp), ("v_codes", _vp),
                 ("k_scales", _vp), ("v_scales", _vp), ("k_gscale", _vp), ("v_gscale", _vp),
-                ("status", _vp)]
+                ("status", _vp), ("flags", ctypes.c_uint32), ("k_mean", _vp)]
 
 
 _CP = ctypes.POINTER(CacheDesc)
@@ -139,9 +141,11 @@ class KVCache:
     """One layer's NVFP4 KV cache; the arrays are torch CUDA tensors owned by this object."""
 
     def __init__(self, batch: int, heads: int, chunk_tokens: int, capacity: int,
-                 q_tokens_max: int = 0, device=None, workspace=None):
+                 q_tokens_max: int = 0, device=None, workspace=None, smooth_k: bool = False,
+                 adaptive_v: bool = False):
         """``workspace``: an optional uint8 CUDA tensor used as this cache's scratch instead of one
-        of its own (caches that run on one stream, one call at a time, may share it)."""
+        of its own (caches that run on one stream, one call at a time, may share it).
+        ``smooth_k`` / ``adaptive_v``: the recipe options K_SMOOTH / V_ADAPTIVE_SCALE."""
         import torch
         self.batch, self.heads, self.chunk_tokens, self.capacity = batch, heads, chunk_tokens, capacity
         dev = torch.device("cuda") if device is None else torch.device(device)
@@ -155,11 +159,15 @@ class KVCache:
         self.k_gscale = torch.zeros(batch, heads, capacity, dtype=torch.float32, device=dev)
         self.v_gscale = torch.zeros(batch, heads, capacity, dtype=torch.float32, device=dev)
         self.status = torch.zeros(4, dtype=torch.int32, device=dev)
+        self.flags = (K_SMOOTH if smooth_k else 0) | (V_ADAPTIVE_SCALE if adaptive_v else 0)
+        self.k_mean = (torch.zeros(batch, heads, capacity, HEAD_DIM, dtype=torch.float32, device=dev)
+                       if smooth_k else None)
         self.desc = CacheDesc(batch, heads, HEAD_DIM, chunk_tokens, capacity,
                               self.k_codes.data_ptr(), self.v_codes.data_ptr(),
                               self.k_scales.data_ptr(), self.v_scales.data_ptr(),
                               self.k_gscale.data_ptr(), self.v_gscale.data_ptr(),
-                              self.status.data_ptr())
+                              self.status.data_ptr(), self.flags,
+                              self.k_mean.data_ptr() if smooth_k else None)
         self._ws = workspace
         self._ws_owned = workspace is None
         self.reserve_workspace(max(q_tokens_max, 1))
@@ -176,8 +184,10 @@ class KVCache:
 
     @property
     def nbytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in (
-            self.k_codes, self.v_codes, self.k_scales, self.v_scales, self.k_gscale, self.v_gscale))
+        arrays = [self.k_codes, self.v_codes, self.k_scales, self.v_scales, self.k_gscale, self.v_gscale]
+        if self.k_mean is not None:
+            arrays.append(self.k_mean)
+        return sum(t.numel() * t.element_size() for t in arrays)
 
     def quantize(self, slot: int, k, v, stream=None) -> None:
         """Quantise bf16 K and V ([B, Lc, H, 128]) of a new chunk into chunk slot ``slot``."""
@@ -195,7 +205,7 @@ class KVCache:
                "nvfp4kv_debug_wait_timeout")
 
     def quantize_launches(self) -> int:
-        """Kernels one ``quantize`` call launches for this cache on the current device (1 or 2)."""
+        """Kernels one ``quantize`` call launches for this cache on the current device (1 to 3)."""
         n = lib().nvfp4kv_quantize_launches(ctypes.byref(self.desc))
         if n < 0:
             raise NvFp4KvError(-n, "nvfp4kv_quantize_launches")

@@ -31,6 +31,8 @@ int check_cache(const nvfp4kv_cache* c) {
   for (const void* p : arrays)
     if (!aligned16(p)) return NVFP4KV_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(c->status) & 3u) return NVFP4KV_ERR_INVALID_ARG;
+  if (c->flags & ~static_cast<uint32_t>(NVFP4KV_K_SMOOTH | NVFP4KV_V_ADAPTIVE_SCALE)) return NVFP4KV_ERR_INVALID_ARG;
+  if ((c->flags & NVFP4KV_K_SMOOTH) && (!c->k_mean || !aligned16(c->k_mean))) return NVFP4KV_ERR_INVALID_ARG;
   return NVFP4KV_OK;
 }
 
@@ -61,6 +63,8 @@ int attention_checked(const nvfp4kv_cache* cache, const void* q_bf16, int32_t q_
   if (out_dtype != NVFP4KV_OUT_F32 && out_dtype != NVFP4KV_OUT_BF16) return NVFP4KV_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale)) return NVFP4KV_ERR_INVALID_ARG;  // NaN
   if (vis.empty()) return NVFP4KV_ERR_INVALID_ARG;
+  // smoothed keys: a 128-key tile may span at most two chunks (the kernel holds two mean terms)
+  if ((cache->flags & NVFP4KV_K_SMOOTH) && cache->chunk_tokens < 128) return NVFP4KV_ERR_UNSUPPORTED;
   if (attention_runs(vis) > kAttnMaxRuns) return NVFP4KV_ERR_UNSUPPORTED;
   int64_t keys = 0;
   for (size_t i = 0; i < vis.size(); ++i) keys += cache->chunk_tokens;
@@ -142,6 +146,7 @@ int nvfp4_kv_quantize_layers(const nvfp4kv_cache* caches, int32_t n_layers, int3
     if (c.batch != c0.batch || c.heads != c0.heads || c.chunk_tokens != c0.chunk_tokens ||
         c.capacity_chunks != c0.capacity_chunks)
       return NVFP4KV_ERR_INVALID_ARG;
+    if (c.flags != 0) return NVFP4KV_ERR_UNSUPPORTED;  // recipe options: one layer at a time
     if (!k_bf16[l] || !v_bf16[l] || !aligned16(k_bf16[l]) || !aligned16(v_bf16[l])) return NVFP4KV_ERR_INVALID_ARG;
   }
   if (chunk_slot < 0 || chunk_slot >= c0.capacity_chunks) return NVFP4KV_ERR_INVALID_ARG;

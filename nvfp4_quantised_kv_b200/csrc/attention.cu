@@ -27,13 +27,16 @@
 //   dequant warps 9-11, 13-15 E2M1 * E4M3 products, exact in fp16, written straight into the
 //                             128B-swizzled UMMA operand layout: K (the B operand of Q K^T,
 //                             K-major) and V (the B operand of P V, MN-major)
-// S is computed in sub-tiles of 64 keys, double-buffered in TMEM per query tile (4 x 64 columns
-// of S, 2 x 128 columns of O): while the softmax warps work on sub-tile h, the tensor core
-// already holds S of sub-tile h + 1, so the softmax never waits on the MMA chain.  The FP32
-// scales stay out of the MMAs: g_K(chunk) multiplies S per column, and g_V(chunk) / max g_V
+// TMEM per query tile q: S of a whole KV tile in columns [128 q, 128 q + 128) (one N = 128 QK
+// chain), O in [256 + 128 q, 384 + 128 q).  The softmax warps take S in two 64-key sub-tiles and
+// store P of sub-tile h over the first 32 columns of its S half; the P V of sub-tile h runs
+// while the softmax works on h + 1, and the next KV tile's QK is issued behind the second P V
+// (MMAs of one thread execute in order, so it cannot overwrite P before P V has read it).  The
+// FP32 scales stay out of the MMAs: g_K(chunk) multiplies S per column, and g_V(chunk) / max g_V
 // multiplies P per column before P is rounded to fp16 (fp16 P and V keep the P V product 8x
 // finer than bf16).  Rows are rescaled lazily: the running max only moves when it grows by more
-// than 2^8.
+// than 2^8.  With smoothed keys (the cache's K-smoothing option) every logit of a chunk's keys
+// also gets scale * q . mu(chunk), computed once per (query row, chunk) from the fp16 Q row.
 //
 // Every mbarrier wait is bounded (%globaltimer); on a time-out the kernel ORs
 // NVFP4KV_ERR_DEVICE_TIMEOUT into the status word, lets in-flight copies and MMAs finish,
@@ -181,6 +184,7 @@ struct AttnParams {
   const uint8_t* v_scales;
   const float* k_g;
   const float* v_g;
+  const float* k_mean;  // smoothed keys: [B*H][C][D] channel means, else null
   void* out;
   float* part;  // partial-result slots: [G][2][kSlotFloats]
   uint32_t* status;
@@ -269,6 +273,32 @@ __device__ __forceinline__ float max_visible_gv(const AttnParams& p, int64_t bh)
   return m > 0.0f ? m : 1.0f;
 }
 
+// q' . mu for one query row: q' is the row's prescaled fp16 copy in the 128B-swizzled Q tile
+// (16-byte chunk j of half hf at position j ^ (row % 8)), mu a chunk's fp32 channel means.
+__device__ __forceinline__ float q_dot_mean(const uint8_t* qrow, int row, const float* mu) {
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int qq = 0; qq < 4; ++qq) {
+    // a quarter's 32 means first (8 independent loads in flight), then its 32 products
+    float4 m[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m[k] = __ldg(reinterpret_cast<const float4*>(mu + qq * 32) + k);
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int hf = qq >> 1, j = (qq & 1) * 4 + jj;  // 16-byte chunk j of half hf
+      const uint4 v = *reinterpret_cast<const uint4*>(qrow + hf * HALF16 + ((j ^ (row & 7)) << 4));
+      const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
+      const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
+      const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&v.z));
+      const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&v.w));
+      const float4 m0 = m[2 * jj], m1 = m[2 * jj + 1];
+      acc[jj] = fmaf(f0.x, m0.x, fmaf(f0.y, m0.y, fmaf(f1.x, m0.z, fmaf(f1.y, m0.w, acc[jj]))));
+      acc[jj] = fmaf(f2.x, m1.x, fmaf(f2.y, m1.y, fmaf(f3.x, m1.z, fmaf(f3.y, m1.w, acc[jj]))));
+    }
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
 __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
   return __vmaxu2(a & 0x7FFF7FFFu, b & 0x7FFF7FFFu);
 }
@@ -325,6 +355,9 @@ __device__ __forceinline__ void dequant_tile(const uint8_t* pk, uint8_t* dst, in
   }
 }
 
+// kSmooth: the cache's keys are smoothed (p.k_mean is set); the plain kernel carries no trace of
+// the per-chunk mean terms.
+template <bool kSmooth>
 __global__ void __launch_bounds__(Cfg::kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ AttnParams p) {
   using C = Cfg;
@@ -472,6 +505,12 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
 
       const float gv_ref = max_visible_gv(p, bh);
       float m_run = -INFINITY, l_run = 0.0f;
+      // smoothed keys: the logit term scale * log2(e) * q . mu of the (at most two) chunks of the
+      // current KV tile, computed when a chunk is first met in this segment
+      int c_lo = -1, c_hi = -1;
+      float b_lo = 0.0f, b_hi = 0.0f;
+      const float b_factor = p.scale_log2 * q_unscale;
+      const float* const mu_bh = kSmooth ? p.k_mean + bh * p.C * D : nullptr;
       const int nh = 2 * ntl;
       for (int hs = 0; hs < nh && ok; ++hs, ++g) {
         const int jj = jjb + (hs >> 1);
@@ -491,6 +530,22 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         // A tile inside one chunk with every key valid takes the uniform path (one logit factor,
         // one cv); any other tile works per column with the same arithmetic.
         const bool uni = info.y != 0;
+        // chunk info.z holds columns [0, info.w), chunk info.z + 1 the valid columns after them
+        if (kSmooth && half == 0) {
+          if (info.z != c_lo) {
+            if (info.z == c_hi) {
+              b_lo = b_hi;
+            } else {
+              b_lo = b_factor * q_dot_mean(qrow, row, mu_bh + info.z * D);
+            }
+            c_lo = info.z;
+          }
+          if (info.w < BN && info.z + 1 != c_hi) {
+            c_hi = info.z + 1;
+            b_hi = b_factor * q_dot_mean(qrow, row, mu_bh + c_hi * D);
+          }
+        }
+        const int jsplit = kSmooth ? info.w - half * SUB : 0;  // first column here in chunk info.z + 1
 
         uint32_t sr[2][32];
         ptx::tmem_ld32(tS, sr[0]);
@@ -504,7 +559,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         float ck = 0.0f, lc = 0.0f;
         if (uni) {
           ck = colK[0] * q_unscale;
-          lc = colL[0];
+          lc = kSmooth ? colL[0] + b_lo : colL[0];
           float m8[8];  // eight independent max chains
 #pragma unroll
           for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
@@ -528,10 +583,18 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
               asm volatile("" ::: "memory");  // keep the table loads next to their use (registers)
               const float4 kk = *reinterpret_cast<const float4*>(colK + 32 * c + i);
               const float4 ll = *reinterpret_cast<const float4*>(colL + 32 * c + i);
-              const float x0 = fmaf(__uint_as_float(sr[c][i]), kk.x * q_unscale, ll.x);
-              const float x1 = fmaf(__uint_as_float(sr[c][i + 1]), kk.y * q_unscale, ll.y);
-              const float x2 = fmaf(__uint_as_float(sr[c][i + 2]), kk.z * q_unscale, ll.z);
-              const float x3 = fmaf(__uint_as_float(sr[c][i + 3]), kk.w * q_unscale, ll.w);
+              float4 l4 = ll;
+              if (kSmooth) {  // the mean term of each column's chunk
+                const int jc = 32 * c + i;  // column within the sub-tile
+                l4.x += jc < jsplit ? b_lo : b_hi;
+                l4.y += jc + 1 < jsplit ? b_lo : b_hi;
+                l4.z += jc + 2 < jsplit ? b_lo : b_hi;
+                l4.w += jc + 3 < jsplit ? b_lo : b_hi;
+              }
+              const float x0 = fmaf(__uint_as_float(sr[c][i]), kk.x * q_unscale, l4.x);
+              const float x1 = fmaf(__uint_as_float(sr[c][i + 1]), kk.y * q_unscale, l4.y);
+              const float x2 = fmaf(__uint_as_float(sr[c][i + 2]), kk.z * q_unscale, l4.z);
+              const float x3 = fmaf(__uint_as_float(sr[c][i + 3]), kk.w * q_unscale, l4.w);
               sr[c][i] = __float_as_uint(x0);
               sr[c][i + 1] = __float_as_uint(x1);
               sr[c][i + 2] = __float_as_uint(x2);
@@ -848,8 +911,10 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
               colK[BN + dt] = valid ? __log2f(gvv) : -INFINITY;
               colK[2 * BN + dt] = valid ? __frcp_rn(gvv) : 0.0f;
               if (dt == 0) {
-                const int uniform = (n == BN) && (key0 / p.Lc == (key0 + BN - 1) / p.Lc);
-                *reinterpret_cast<int4*>(smem + C::oInfo + 16 * ct) = make_int4(n, uniform, 0, 0);
+                const int c0 = key0 / p.Lc;
+                const int uniform = (n == BN) && (c0 == (key0 + BN - 1) / p.Lc);
+                const int split = (c0 + 1) * p.Lc - key0;  // first column in chunk c0 + 1
+                *reinterpret_cast<int4*>(smem + C::oInfo + 16 * ct) = make_int4(n, uniform, c0, split < n ? split : BN);
               }
             }
             ptx::fence_proxy_async_smem();
@@ -1101,6 +1166,7 @@ int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, in
   prm.v_scales = c.v_scales;
   prm.k_g = c.k_gscale;
   prm.v_g = c.v_gscale;
+  prm.k_mean = (c.flags & NVFP4KV_K_SMOOTH) ? c.k_mean : nullptr;
   prm.out = out;
   prm.part = static_cast<float*>(workspace);
   prm.status = c.status;
@@ -1152,10 +1218,17 @@ int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, in
     return NVFP4KV_ERR_WORKSPACE;
 
   const cudaError_t ae = g_attn_attr.run([] {
-    return cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(attention_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+    return e;
   });
   if (ae != cudaSuccess) return NVFP4KV_ERR_CUDA;
-  attention_kernel<<<prm.pl.G, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tm, prm);
+  if (prm.k_mean)
+    attention_kernel<true><<<prm.pl.G, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tm, prm);
+  else
+    attention_kernel<false><<<prm.pl.G, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tm, prm);
   if (cudaGetLastError() != cudaSuccess) return NVFP4KV_ERR_CUDA;
   if (splits) {
     cudaLaunchConfig_t cfg = {};

@@ -16,8 +16,9 @@ namespace nvfp4kv {
 namespace {
 
 __global__ void dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                               const float* __restrict__ gscale, int BH, int Lc, int C,
-                               int first_slot, int n_slots, int as_bf16, float* __restrict__ out) {
+                               const float* __restrict__ gscale, const float* __restrict__ kmean, int BH,
+                               int Lc, int C, int first_slot, int n_slots, int as_bf16,
+                               float* __restrict__ out) {
   const int64_t span = static_cast<int64_t>(n_slots) * Lc;
   const int64_t total = static_cast<int64_t>(BH) * span * 16;
   const int64_t T = static_cast<int64_t>(C) * Lc;
@@ -52,6 +53,11 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t*
       o[2 * i] = __fmul_rn(lo, g);
       o[2 * i + 1] = __fmul_rn(hi, g);
     }
+    if (kmean) {  // a smoothed key: x_hat' + mu of its chunk
+      const float* mu = kmean + (bh * C + t / Lc) * kHeadDim + c16 * 8;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = __fadd_rn(o[i], mu[i]);
+    }
     float4* dst = reinterpret_cast<float4*>(out + (bh * span + tt) * kHeadDim + c16 * 8);
     dst[0] = make_float4(o[0], o[1], o[2], o[3]);
     dst[1] = make_float4(o[4], o[5], o[6], o[7]);
@@ -83,7 +89,9 @@ cudaError_t launch_dequantize(const nvfp4kv_cache& c, int which, int first_slot,
   if (blocks < 1) blocks = 1;
   dequant_kernel<<<blocks, 256, 0, stream>>>(is_k ? c.k_codes : c.v_codes,
                                              is_k ? c.k_scales : c.v_scales,
-                                             is_k ? c.k_gscale : c.v_gscale, BH, c.chunk_tokens,
+                                             is_k ? c.k_gscale : c.v_gscale,
+                                             is_k && (c.flags & NVFP4KV_K_SMOOTH) ? c.k_mean : nullptr, BH,
+                                             c.chunk_tokens,
                                              c.capacity_chunks, first_slot, n_slots, is_k ? 1 : 0,
                                              out);
   return cudaGetLastError();

@@ -49,10 +49,12 @@ struct QuantArgs {
   uint8_t* codes[2];
   uint8_t* scales[2];
   float* gscale[2];
-  uint32_t* partial;  // [2][B*H][parts], bf16 bit pattern of a partial max|x|
+  uint32_t* partial;  // [2][B*H][parts], bf16 bit pattern of a partial max|x| (fp32 bits on the recipe path)
+  const float* k_mean;  // recipe path with K-smoothing: the cache's k_mean, else null
   int64_t token_stride;
   int64_t T;  // tokens per (b, h) in the cache
   int B, H, L, C, slot, parts;
+  uint32_t flags;  // recipe options (NVFP4KV_K_SMOOTH, NVFP4KV_V_ADAPTIVE_SCALE)
 };
 
 __device__ __forceinline__ uint4 ld_row16(const uint16_t* p) {
@@ -225,6 +227,302 @@ __global__ void __launch_bounds__(kThreads, 6) quantize_kernel(const __grid_cons
     const int t = t_begin + u * (kThreads / 16) + sub;
     encode_store(w[u], enc, rtab, t < t_end, codes + static_cast<int64_t>(t) * kCodeBytes,
                  scales + static_cast<int64_t>(t) * kScaleBytes, lane);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Recipe path, taken by caches with recipe options: K-smoothing of K and adaptive {4, 6}
+// block-scale targets of V (reading note, "The inference infrastructure": both applied within
+// each chunk; "Engineering details of NVFP4 training": candidate scale magnitudes {4, 6}).
+//   key_mean_kernel       one CTA per (32 channels, b, h): TMA brings 64-token slices of the
+//                         chunk's keys into a ring in shared memory and one warp adds them up, a
+//                         lane per channel, in fp64 in token order; mu = fp32(sum / L) is written
+//                         to the slot's k_mean.  (The sum is one dependent chain per channel:
+//                         its order is part of the definition.)
+//   recipe_amax_kernel    amax_kernel over x - mu for a smoothed K (fp32 magnitudes); the
+//                         partials hold fp32 bit patterns for both tensors.
+//   recipe_encode_kernel  quantize_kernel from x - mu for a smoothed K; for V with adaptive
+//                         scales each block is encoded for both scale targets and keeps the one
+//                         with the smaller fp64 squared error, ties keeping 6.
+constexpr int kMeanTok = 64;    // tokens per ring stage
+constexpr int kMeanCh = 32;     // channels per CTA (64 bytes of each token row)
+constexpr int kMeanStages = 8;  // 8 x 4 KB in flight per CTA
+
+struct MeanArgs {
+  float* k_mean;
+  uint32_t* status;
+  int H, L, C, slot;
+};
+
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity) {
+  uint64_t t0 = 0;
+  int it = 0;
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    const uint64_t now = ptx::globaltimer_ns();
+    if (it++ == 0) t0 = now;
+    if (now - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(64) key_mean_kernel(const __grid_constant__ CUtensorMap tm,
+                                                      const __grid_constant__ MeanArgs a) {
+  __shared__ __align__(128) uint16_t ring[kMeanStages][kMeanTok * kMeanCh];
+  __shared__ __align__(8) uint64_t full[kMeanStages], empty[kMeanStages];
+  __shared__ int s_issued;
+  const int cg = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (a.L + kMeanTok - 1) / kMeanTok;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMeanStages; ++i) {
+      ptx::mbar_init(ptx::smem_u32(&full[i]), 1);
+      ptx::mbar_init(ptx::smem_u32(&empty[i]), 1);
+    }
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  bool ok = true;
+  if (warp == 1) {
+    // producer: one TMA box (64 tokens x 32 channels) per stage; a stage is reused once the
+    // summing warp has released it
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < n_tiles; ++i) {
+        const int st = i % kMeanStages;
+        if (i >= kMeanStages && !wait_phase(ptx::smem_u32(&empty[st]), ((i / kMeanStages) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        ptx::mbar_arrive_expect_tx(ptx::smem_u32(&full[st]), kMeanTok * kMeanCh * 2);
+        ptx::tma_load_4d(ptx::smem_u32(ring[st]), &tm, cg * kMeanCh, h, i * kMeanTok, b, ptx::smem_u32(&full[st]));
+        ++issued;
+      }
+      s_issued = issued;
+    }
+  } else {
+    // one lane per channel: the fp64 sum in token order
+    double sum = 0.0;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int st = i % kMeanStages;
+      ok = __all_sync(0xFFFFFFFFu, wait_phase(ptx::smem_u32(&full[st]), (i / kMeanStages) & 1));
+      if (!ok) break;
+      const int n = min(kMeanTok, a.L - i * kMeanTok);
+      const uint16_t* col = ring[st] + lane;
+      if (n == kMeanTok) {
+        // a full stage: every shared-memory load first, then the dependent adds in token order
+        uint16_t v[kMeanTok];
+        const uint32_t base = ptx::smem_u32(col);
+#pragma unroll
+        for (int t = 0; t < kMeanTok; ++t)  // volatile: all 64 loads stay ahead of the adds
+          asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v[t]) : "r"(base + t * kMeanCh * 2));
+#pragma unroll
+        for (int t = 0; t < kMeanTok; ++t) sum += static_cast<double>(__uint_as_float(static_cast<uint32_t>(v[t]) << 16));
+      } else {
+        for (int t = 0; t < n; ++t) sum += static_cast<double>(__uint_as_float(static_cast<uint32_t>(col[t * kMeanCh]) << 16));
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty[st]));
+    }
+    if (ok)
+      a.k_mean[(static_cast<int64_t>(bh) * a.C + a.slot) * kHeadDim + cg * kMeanCh + lane] =
+          __double2float_rn(sum / static_cast<double>(a.L));
+  }
+  if (!ok && (lane == 0)) atomicOr(a.status, kStatusTimeout);
+  __syncthreads();
+  if (threadIdx.x == 32) {
+    // after a time-out some copies may still be in flight: let them land (bounded) before the
+    // CTA's shared memory goes away
+    for (int i = max(0, s_issued - kMeanStages); i < s_issued; ++i)
+      if (!wait_phase(ptx::smem_u32(&full[i % kMeanStages]), (i / kMeanStages) & 1)) break;
+  }
+}
+
+// this thread's 8 elements of one token row as fp32: x, or x - mu (one fp32 subtraction each)
+__device__ __forceinline__ void row_values(uint4 w, const float (&mu)[8], bool smooth, float (&y)[8]) {
+  const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    y[2 * i] = __uint_as_float(wv[i] << 16);
+    y[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+  }
+  if (smooth) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = __fsub_rn(y[i], mu[i]);
+  }
+}
+
+__device__ __forceinline__ void load_mu(const QuantArgs& a, int bh, int tensor, bool& smooth, float (&mu)[8]) {
+  smooth = tensor == 0 && (a.flags & NVFP4KV_K_SMOOTH);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mu[i] = 0.0f;
+  if (smooth) {
+    const float* m = a.k_mean + (static_cast<int64_t>(bh) * a.C + a.slot) * kHeadDim + (threadIdx.x & 15) * 8;
+    const float4 m0 = *reinterpret_cast<const float4*>(m), m1 = *reinterpret_cast<const float4*>(m + 4);
+    mu[0] = m0.x; mu[1] = m0.y; mu[2] = m0.z; mu[3] = m0.w;
+    mu[4] = m1.x; mu[5] = m1.y; mu[6] = m1.z; mu[7] = m1.w;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 4) recipe_amax_kernel(const __grid_constant__ QuantArgs a) {
+  const int part = blockIdx.x, bh = blockIdx.y, tensor = blockIdx.z;
+  const int b = bh / a.H, h = bh % a.H;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int t_begin = part * kPartTokens;
+  const int t_end = min(a.L, t_begin + kPartTokens);
+  const int sub = threadIdx.x >> 4;
+  const uint16_t* x = a.x[tensor] + static_cast<int64_t>(b) * a.L * a.token_stride +
+                      static_cast<int64_t>(h) * kHeadDim + (threadIdx.x & 15) * 8;
+  uint4 w[kPasses];
+#pragma unroll
+  for (int u = 0; u < kPasses; ++u) {
+    const int t = t_begin + u * (kThreads / 16) + sub;
+    w[u] = t < t_end ? ld_row16(x + static_cast<int64_t>(t) * a.token_stride) : make_uint4(0, 0, 0, 0);
+  }
+  bool smooth;
+  float mu[8];
+  load_mu(a, bh, tensor, smooth, mu);
+  float m = 0.0f;
+#pragma unroll
+  for (int u = 0; u < kPasses; ++u) {
+    const int t = t_begin + u * (kThreads / 16) + sub;
+    float y[8];
+    row_values(w[u], mu, smooth, y);
+    if (t < t_end)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(y[i]));
+  }
+  uint32_t mb = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));  // non-negative floats order as integers
+  __shared__ uint32_t red[kWarps];
+  if (lane == 0) red[warp] = mb;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t r = 0;
+#pragma unroll
+    for (int i = 0; i < kWarps; ++i) r = max(r, red[i]);
+    a.partial[(static_cast<int64_t>(tensor) * a.B * a.H + bh) * a.parts + part] = r;
+  }
+}
+
+// E2M1 magnitude code (0..7) -> value {0, 0.5, 1, 1.5, 2, 3, 4, 6}
+__device__ __forceinline__ double e2m1_value(uint32_t nib) {
+  const uint32_t m = nib & 7u;
+  const double v = m < 4 ? 0.5 * m : static_cast<double>(1u << ((m - 2) >> 1)) * ((m & 1u) ? 1.5 : 1.0);
+  return (nib & 8u) ? -v : v;
+}
+
+// E2M1 codes of y * r (8 elements, element 2j in the low nibble of byte j); 0 when r is 0
+__device__ __forceinline__ uint32_t codes8f(const float (&y)[8], float r) {
+  if (r == 0.0f) return 0u;
+  float z[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) z[i] = __fmul_rn(y[i], r);
+  return ptx::f32x8_to_e2m1x8(z);
+}
+
+// squared error terms (y_i - E2M1(q_i) * s * g)^2 of this lane's 8 elements, each operation
+// rounded once in fp64
+__device__ __forceinline__ void sq_terms(const float (&y)[8], uint32_t q, uint32_t s_code, float g, double (&sq)[8]) {
+  const double sv = static_cast<double>(ptx::e4m3_to_f32(s_code)), gd = static_cast<double>(g);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const double xh = __dmul_rn(__dmul_rn(e2m1_value((q >> (4 * i)) & 0xFu), sv), gd);
+    const double diff = __dadd_rn(static_cast<double>(y[i]), -xh);
+    sq[i] = __dmul_rn(diff, diff);
+  }
+}
+
+// the block's squared error, summed over its 16 elements in order: the even lane of the pair
+// holds elements 0-7, the odd lane 8-15 and continues from the even lane's partial sum
+__device__ __forceinline__ double block_sq_error(const double (&sq)[8], int lane) {
+  double acc = 0.0;
+  if ((lane & 1) == 0)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc = __dadd_rn(acc, sq[i]);
+  const double from_even = __shfl_xor_sync(0xFFFFFFFFu, acc, 1);
+  if (lane & 1) {
+    acc = from_even;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc = __dadd_rn(acc, sq[i]);
+  }
+  return acc;  // complete on the odd lane
+}
+
+__global__ void __launch_bounds__(kThreads, 2) recipe_encode_kernel(const __grid_constant__ QuantArgs a) {
+  const int part = blockIdx.x, bh = blockIdx.y, tensor = blockIdx.z;
+  const int b = bh / a.H, h = bh % a.H;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t_begin = part * kEncTokens;
+  const int t_end = min(a.L, t_begin + kEncTokens);
+  const int sub = threadIdx.x >> 4;
+  const uint16_t* x = a.x[tensor] + static_cast<int64_t>(b) * a.L * a.token_stride +
+                      static_cast<int64_t>(h) * kHeadDim + (threadIdx.x & 15) * 8;
+  uint4 w[kEncPasses];
+#pragma unroll
+  for (int u = 0; u < kEncPasses; ++u) {
+    const int t = t_begin + u * (kThreads / 16) + sub;
+    w[u] = t < t_end ? ld_row16(x + static_cast<int64_t>(t) * a.token_stride) : make_uint4(0, 0, 0, 0);
+  }
+  bool smooth;
+  float mu[8];
+  load_mu(a, bh, tensor, smooth, mu);
+  const bool adaptive = tensor == 1 && (a.flags & NVFP4KV_V_ADAPTIVE_SCALE);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  __shared__ float s_g;
+  if (warp == 0) {
+    const uint32_t* p = a.partial + (static_cast<int64_t>(tensor) * a.B * a.H + bh) * a.parts;
+    uint32_t m = 0;
+    for (int i = lane; i < a.parts; i += 32) m = max(m, p[i]);
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if (lane == 0) {
+      const float A = __uint_as_float(m);
+      const float g = (A == 0.0f) ? 0.0f : __fdiv_rn(A, 2688.0f);
+      s_g = g;
+      if (part == 0) a.gscale[tensor][static_cast<int64_t>(bh) * a.C + a.slot] = g;
+    }
+  }
+  __shared__ float rtab[128];
+  __syncthreads();
+  const Encoder enc = make_encoder(s_g, rtab, threadIdx.x, kThreads);
+  Encoder enc4 = enc;  // scale target 4: a_b / (4 g), with 4 g exact
+  enc4.d = __fmul_rn(4.0f, enc.g);
+  enc4.y = enc.g != 0.0f ? __frcp_rn(enc4.d) : 0.0f;
+  enc4.fast = enc.g != 0.0f && enc4.d >= 0x1p-126f && enc4.y >= 0x1p-126f && enc4.y < 0x1p127f;
+  __syncthreads();
+
+  const int64_t row0 = static_cast<int64_t>(bh) * a.T + static_cast<int64_t>(a.slot) * a.L;
+  uint8_t* codes = a.codes[tensor] + row0 * kCodeBytes + (lane & 15) * 4;
+  uint8_t* scales = a.scales[tensor] + row0 * kScaleBytes + ((lane & 15) >> 1);
+#pragma unroll
+  for (int u = 0; u < kEncPasses; ++u) {
+    const int t = t_begin + u * (kThreads / 16) + sub;
+    float y[8];
+    row_values(w[u], mu, smooth, y);
+    float am = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(y[i]));
+    const float ab = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+    uint32_t s_code = block_scale_code(ab, enc);
+    uint32_t qc = codes8f(y, rtab[s_code & 0x7F]);
+    if (adaptive) {  // warp-uniform: the tensor is the CTA's
+      const uint32_t s4 = block_scale_code(ab, enc4);
+      const uint32_t q4 = codes8f(y, rtab[s4 & 0x7F]);
+      double sq6[8], sq4[8];
+      sq_terms(y, qc, s_code, enc.g, sq6);
+      sq_terms(y, q4, s4, enc.g, sq4);
+      const double e6 = block_sq_error(sq6, lane), e4 = block_sq_error(sq4, lane);
+      const bool pick4 = __shfl_sync(0xFFFFFFFFu, e4 < e6 ? 1 : 0, lane | 1) != 0;  // the odd lane decides
+      if (pick4) {
+        s_code = s4;
+        qc = q4;
+      }
+    }
+    if (t < t_end) {
+      *reinterpret_cast<uint32_t*>(codes + static_cast<int64_t>(t) * kCodeBytes) = qc;
+      if ((lane & 1) == 0) scales[static_cast<int64_t>(t) * kScaleBytes] = static_cast<uint8_t>(s_code);
+    }
   }
 }
 
@@ -646,16 +944,15 @@ cudaError_t launch_cluster(const nvfp4kv_cache& c, int slot, const uint16_t* k, 
 
 }  // namespace
 
-int quantize_launches(const nvfp4kv_cache& c) { return cluster_plan(c).cl > 0 ? 1 : 2; }
+int quantize_launches(const nvfp4kv_cache& c) {
+  if (c.flags != 0) return (c.flags & NVFP4KV_K_SMOOTH) ? 3 : 2;
+  return cluster_plan(c).cl > 0 ? 1 : 2;
+}
 
-cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
-                            int64_t token_stride, void* workspace, cudaStream_t stream) {
-  const ClusterPlan pl = cluster_plan(c);
-  if (pl.cl > 0) {
-    bool launched = false;
-    const cudaError_t e = launch_cluster(c, slot, k, v, token_stride, pl, stream, &launched);
-    if (launched || e != cudaSuccess) return e;
-  }
+namespace {
+
+QuantArgs two_pass_args(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
+                        int64_t token_stride, void* workspace) {
   QuantArgs a;
   a.x[0] = k;
   a.x[1] = v;
@@ -666,6 +963,7 @@ cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k,
   a.gscale[0] = c.k_gscale;
   a.gscale[1] = c.v_gscale;
   a.partial = static_cast<uint32_t*>(workspace);
+  a.k_mean = c.k_mean;
   a.token_stride = token_stride;
   a.T = static_cast<int64_t>(c.capacity_chunks) * c.chunk_tokens;
   a.B = c.batch;
@@ -674,14 +972,16 @@ cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k,
   a.C = c.capacity_chunks;
   a.slot = slot;
   a.parts = quantize_parts(c.batch, c.heads, c.chunk_tokens);
-  const dim3 grid(a.parts, c.batch * c.heads, 2);
-  amax_kernel<<<grid, kThreads, 0, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  // The encode grid is a programmatic dependent of the amax grid: it launches while the amax grid
-  // drains and waits (griddepcontrol.wait) only before it reads the partial maxima.
+  a.flags = c.flags;
+  return a;
+}
+
+// The encode grid of the two-pass paths, a programmatic dependent of the amax grid: it launches
+// while the amax grid drains and waits (griddepcontrol.wait) only before it reads the maxima.
+template <typename Kernel>
+cudaError_t launch_encode_dependent(Kernel kernel, const QuantArgs& a, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((c.chunk_tokens + kEncTokens - 1) / kEncTokens, c.batch * c.heads, 2);
+  cfg.gridDim = dim3((a.L + kEncTokens - 1) / kEncTokens, a.B * a.H, 2);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -689,7 +989,59 @@ cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, quantize_kernel, a);
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
+cudaError_t launch_quantize_recipe(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
+                                   int64_t token_stride, void* workspace, cudaStream_t stream) {
+  const QuantArgs a = two_pass_args(c, slot, k, v, token_stride, workspace);
+  if (c.flags & NVFP4KV_K_SMOOTH) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (!encode) return cudaErrorNotSupported;
+    CUtensorMap tm;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(c.heads),
+                                static_cast<cuuint64_t>(c.chunk_tokens), static_cast<cuuint64_t>(c.batch)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHeadDim) * 2, static_cast<cuuint64_t>(token_stride) * 2,
+                                   static_cast<cuuint64_t>(c.chunk_tokens) * token_stride * 2};
+    const cuuint32_t box[4] = {kMeanCh, 1, kMeanTok, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (encode(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(k), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    MeanArgs m;
+    m.k_mean = c.k_mean;
+    m.status = c.status;
+    m.H = c.heads;
+    m.L = c.chunk_tokens;
+    m.C = c.capacity_chunks;
+    m.slot = slot;
+    key_mean_kernel<<<dim3(kHeadDim / kMeanCh, c.batch * c.heads), 64, 0, stream>>>(tm, m);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  recipe_amax_kernel<<<dim3(a.parts, c.batch * c.heads, 2), kThreads, 0, stream>>>(a);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_encode_dependent(recipe_encode_kernel, a, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
+                            int64_t token_stride, void* workspace, cudaStream_t stream) {
+  if (c.flags != 0) return launch_quantize_recipe(c, slot, k, v, token_stride, workspace, stream);
+  const ClusterPlan pl = cluster_plan(c);
+  if (pl.cl > 0) {
+    bool launched = false;
+    const cudaError_t e = launch_cluster(c, slot, k, v, token_stride, pl, stream, &launched);
+    if (launched || e != cudaSuccess) return e;
+  }
+  const QuantArgs a = two_pass_args(c, slot, k, v, token_stride, workspace);
+  amax_kernel<<<dim3(a.parts, c.batch * c.heads, 2), kThreads, 0, stream>>>(a);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_encode_dependent(quantize_kernel, a, stream);
 }
 
 PerDeviceOnce g_ticket_occ;

@@ -164,3 +164,24 @@ def test_strerror_covers_every_code(L):
     for code in range(6):
         assert nk.strerror(code) != "unknown status"
     assert nk.strerror(99) == "unknown status"
+
+
+def test_recipe_flags_are_checked_before_any_launch(L):
+    bad = _desc(flags=4)  # an unknown option bit
+    assert L.nvfp4_kv_quantize(ctypes.byref(bad), 0, 0x80000, 0x90000, 256, 0xA0000, 1 << 20, None) == nk.ERR_INVALID_ARG
+    no_mean = _desc(flags=nk.K_SMOOTH)  # smoothing without its mean array
+    assert L.nvfp4_kv_quantize(ctypes.byref(no_mean), 0, 0x80000, 0x90000, 256, 0xA0000, 1 << 20,
+                               None) == nk.ERR_INVALID_ARG
+    odd = _desc(flags=nk.K_SMOOTH, k_mean=0xB0008)  # misaligned mean array
+    assert L.nvfp4_kv_quantize(ctypes.byref(odd), 0, 0x80000, 0x90000, 256, 0xA0000, 1 << 20, None) == nk.ERR_INVALID_ARG
+    # smoothed attention needs chunks of at least 128 tokens (a tile spans at most two chunks)
+    short = _desc(flags=nk.K_SMOOTH, k_mean=0xB0000, chunk_tokens=64)
+    out = (ctypes.c_int32 * 1)()
+    rc = L.nvfp4_kv_attention(ctypes.byref(short), 0x80000, 64, 256, 1, 1, 2, 0.0, 0xC0000, 0, 0xA0000,
+                              1 << 24, None)
+    assert rc == nk.ERR_UNSUPPORTED
+    del out
+    # the single-launch multi-layer quantiser takes plain caches only
+    pair = (nk.CacheDesc * 2)(_desc(), _desc(flags=nk.V_ADAPTIVE_SCALE))
+    ks = (ctypes.c_void_p * 2)(0x80000, 0x80000)
+    assert L.nvfp4_kv_quantize_layers(pair, 2, 0, ks, ks, 256, 0xA0000, 1 << 20, None) == nk.ERR_UNSUPPORTED
