@@ -1,9 +1,11 @@
 /* Host check of the quantiser's block-scale quotient shortcut.  For a chunk maximum A (a bf16
- * value), d = RN(6 * RN(A / 2688)); the kernel takes q = RN(a * y) with y = RN(1 / d), then
- * q' = RN(q + RN(a - q * d) * y) (two FMAs), instead of RN(a / d), whenever d and y are normal
- * and a >= 2^-100.  Only the E4M3 code of the quotient is stored, so the check compares codes:
- * E4M3 round-to-nearest-even with saturation at 448, found by nearest-value search.
- * Usage: block_scale_quotient N_CHUNK_MAXIMA GUARD(0|1); prints "tested T mismatches M". */
+ * value), d = RN(T * RN(A / 2688)) for the scale target T (6, or 4 for the adaptive candidate);
+ * the kernel takes q = RN(a * y) with y = RN(1 / d), then q' = RN(q + RN(a - q * d) * y) (two
+ * FMAs), instead of RN(a / d), whenever d and y are normal and a >= 2^-100.  Only the E4M3 code
+ * of the quotient is stored, so the check compares codes: E4M3 round-to-nearest-even with
+ * saturation at 448, found by nearest-value search.
+ * Usage: block_scale_quotient N_CHUNK_MAXIMA GUARD(0|1) [T]; N_CHUNK_MAXIMA = 0 takes every
+ * positive finite bf16 chunk maximum; prints "tested T mismatches M". */
 #include <math.h>
 #include <stdint.h>
 #include <stdio.h>
@@ -36,8 +38,11 @@ static int e4m3_rne(float q) {
 }
 
 int main(int argc, char** argv) {
-  const int n_max = argc > 1 ? atoi(argv[1]) : 600;
+  const int n_arg = argc > 1 ? atoi(argv[1]) : 600;
   const int guard = argc > 2 ? atoi(argv[2]) : 1;
+  const float target = argc > 3 ? (float)atof(argv[3]) : 6.0f;
+  const int all = n_arg == 0;
+  const int n_max = all ? 0x7F7F : n_arg;
   long tested = 0, mism = 0;
   uint64_t st = 88172645463325252ull;
   for (int ai = 0; ai < n_max; ++ai) {
@@ -46,10 +51,11 @@ int main(int argc, char** argv) {
     st ^= st << 17;
     uint16_t abits = (uint16_t)(st % 0x7F80u);
     if (ai < 64) abits = (uint16_t)(0x0001 + ai * 0x01FF); /* the small end, subnormals included */
+    if (all) abits = (uint16_t)(ai + 1);                     /* 0x0001 .. 0x7F7F: every one */
     const float A = bf16(abits);
     if (A == 0.0f) continue;
     const float g = A / 2688.0f;
-    const float d = 6.0f * g;
+    const float d = target * g;
     const float y = 1.0f / d;
     if (!isnormal(d) || !isnormal(y)) continue; /* the kernel divides for these chunks */
     for (uint32_t b = 1; b <= abits; ++b) {

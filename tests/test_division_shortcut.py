@@ -20,8 +20,9 @@ def exe(tmp_path_factory):
     return out
 
 
-def _run(exe, n, guard):
-    text = subprocess.run([exe, str(n), str(guard)], check=True, capture_output=True, text=True).stdout
+def _run(exe, n, guard, target=6):
+    text = subprocess.run([exe, str(n), str(guard), str(target)], check=True, capture_output=True,
+                          text=True).stdout
     _, tested, _, mism = text.split()
     return int(tested), int(mism)
 
@@ -35,3 +36,12 @@ def test_shortcut_matches_division_codes_where_the_kernel_uses_it(exe):
 def test_the_tiny_block_guard_is_needed(exe):
     _, mism = _run(exe, 600, 0)
     assert mism > 0
+
+
+@pytest.mark.parametrize("target", [6, 4])
+def test_shortcut_matches_division_codes_for_every_bf16_chunk_maximum(exe, target):
+    # every positive finite bf16 chunk maximum A and every bf16 block maximum a <= A, for the
+    # scale target 6 and the adaptive candidate's target 4
+    tested, mism = _run(exe, 0, 1, target)
+    assert tested > 400_000_000
+    assert mism == 0
