@@ -35,7 +35,7 @@
 // FP32 scales stay out of the MMAs: g_K(chunk) multiplies S per column, and g_V(chunk) / max g_V
 // multiplies P per column before P is rounded to fp16 (fp16 P and V keep the P V product 8x
 // finer than bf16).  Rows are rescaled lazily: the running max only moves when it grows by more
-// than 2^8.  With smoothed keys (the cache's K-smoothing option) every logit of a chunk's keys
+// than 2^14 (so P~ stays below 2^14 * 2^(rounding), inside fp16's range).  With smoothed keys (the cache's K-smoothing option) every logit of a chunk's keys
 // also gets scale * q . mu(chunk), computed once per (query row, chunk) from the fp16 Q row.
 //
 // Every mbarrier wait is bounded (%globaltimer); on a time-out the kernel ORs
@@ -604,10 +604,12 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
           mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         }
         // Lazy rescale: the reference m only moves (to a whole number, so the rescale is an exact
-        // power of two) when the row maximum exceeds it by more than 2^8.  The O rescale uses
+        // power of two) when the row maximum exceeds it by more than 2^14; P~ = 2^(x - m) then stays
+        // below 2^14 (fp16 holds up to 65504), and an O rescale, which waits for the tile's P V,
+        // is rare.  The O rescale uses
         // warp-collective TMEM accesses, so it runs for the whole warp when any row moved
         // (alpha = 1 for the rows that did not).
-        const bool grow = mx > m_run + 8.0f;
+        const bool grow = mx > m_run + 14.0f;
         if (__any_sync(0xFFFFFFFFu, grow)) {
           const float m_new = grow ? ceilf(mx) : m_run;
           const float alpha = grow ? ptx::ex2(m_run - m_new) : 1.0f;  // 0 while m is -inf
