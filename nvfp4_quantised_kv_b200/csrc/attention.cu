@@ -948,83 +948,96 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
 //   m* = max_k m_k;  O = sum_k O_k 2^(m_k - m*);  l = sum_k l_k 2^(m_k - m*);  out = O g_ref / l
 // (the m_k are whole numbers, so every factor is an exact power of two).  Launched as a
 // programmatic dependent of the attention grid: it waits for that grid before reading partials.
-constexpr int kCombineRows = 16;
+constexpr int kCombineRows = 16;  // rows of one split item per CTA: 8 warps x 2 rows
+constexpr int kCombineParts = 4;  // parts merged with all their loads in flight at once
 
-__global__ void __launch_bounds__(32 * kCombineRows) combine_kernel(const __grid_constant__ AttnParams p) {
+// One split item's 16 rows: the parts' (m, l, O) rows are all loaded before any is used, so a row
+// costs one round trip to L2 (items split into more than kCombineParts parts loop).
+__global__ void __launch_bounds__(32 * kCombineRows / 2) combine_kernel(const __grid_constant__ AttnParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const Plan& pl = p.pl;
   const int bnd = blockIdx.x + 1;
-  const int64_t u = plan_cut(pl, bnd);
-  if (u >= pl.units || u % pl.NT == 0) return;
-  const int64_t item = u / pl.NT, istart = item * pl.NT, iend = istart + pl.NT;
-  const int bhi = static_cast<int>(item / pl.ipb), k = static_cast<int>(item % pl.ipb);
-  const int m0 = 2 * k * BM, nq = (2 * k + 1 < pl.n_qt) ? 2 : 1;
-  const int r = blockIdx.y * kCombineRows + (threadIdx.x >> 5);  // query row of the item
-  if (blockIdx.y * kCombineRows >= nq * BM || m0 + blockIdx.y * kCombineRows >= p.Lq) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ int slots[kMaxCtas];
   __shared__ int n_slots;
-  if (threadIdx.x == 0) {
+  __shared__ int s_item;
+  if (warp == 0) {
+    // the item split at cut bnd and the CTAs whose ranges meet it: lane i looks at CTA bnd - 1 + i
+    const int64_t u = plan_cut(pl, bnd);
+    const bool split = u < pl.units && u % pl.NT != 0;
+    const int64_t item = u / pl.NT, istart = item * pl.NT, iend = istart + pl.NT;
     int n = 0;
-    if (plan_cut(pl, bnd - 1) <= istart) {  // otherwise an earlier boundary lies inside this item
-      for (int c = bnd - 1; c < pl.G; ++c) {
-        const int64_t cs = plan_cut(pl, c), ce = plan_cut(pl, c + 1);
-        if (cs >= iend) break;
-        if (ce <= istart || cs == ce) continue;
-        slots[n++] = 2 * c + (cs < istart ? 1 : 0);
+    // only the item's first cut merges it (an earlier cut inside the same item leaves it alone)
+    if (split && plan_cut(pl, bnd - 1) <= istart) {
+      for (int base = bnd - 1; base < pl.G; base += 32) {
+        const int c = base + lane;
+        const int64_t cs = c < pl.G ? plan_cut(pl, c) : iend, ce = c < pl.G ? plan_cut(pl, c + 1) : iend;
+        const bool meets = c < pl.G && cs < iend && ce > istart && cs < ce;
+        const unsigned mask = __ballot_sync(0xFFFFFFFFu, meets);
+        if (meets) slots[n + __popc(mask & ((1u << lane) - 1u))] = 2 * c + (cs < istart ? 1 : 0);
+        n += __popc(mask);
+        if (__any_sync(0xFFFFFFFFu, c < pl.G && cs >= iend)) break;
       }
     }
-    n_slots = n;
+    if (lane == 0) {
+      n_slots = n;
+      s_item = static_cast<int>(item);
+    }
   }
   __syncthreads();
   const int ns = n_slots;
-  const int qrow = m0 + r;
-  if (ns == 0 || r >= nq * BM || qrow >= p.Lq) return;
-  const int lane = threadIdx.x & 31;
+  if (ns == 0) return;
+  const int item = s_item;
+  const int bhi = item / pl.ipb, k = item % pl.ipb;
+  const int m0 = 2 * k * BM, nq = (2 * k + 1 < pl.n_qt) ? 2 : 1;
   const int b = bhi / p.H, h = bhi % p.H;
-  float mstar = -INFINITY;
-  for (int i = lane; i < ns; i += 32)
-    mstar = fmaxf(mstar, p.part[static_cast<int64_t>(slots[i]) * kSlotFloats + QT * BM * D + r]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xFFFFFFFFu, mstar, o));
-  float lsum = 0.0f;
-  for (int i = lane; i < ns; i += 32) {
-    const float* sp = p.part + static_cast<int64_t>(slots[i]) * kSlotFloats;
-    lsum += ptx::ex2(sp[QT * BM * D + r] - mstar) * sp[QT * BM * D + QT * BM + r];
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xFFFFFFFFu, lsum, o);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i0 = 0; i0 < ns; i0 += 4) {
-    float4 ov[4];
-    float wv[4];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {  // four parts' loads in flight
-      const int i = i0 + t < ns ? i0 + t : i0;
-      const float* sp = p.part + static_cast<int64_t>(slots[i]) * kSlotFloats;
-      ov[t] = reinterpret_cast<const float4*>(sp + r * D)[lane];
-      wv[t] = i0 + t < ns ? ptx::ex2(sp[QT * BM * D + r] - mstar) : 0.0f;
-    }
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      acc.x = fmaf(wv[t], ov[t].x, acc.x);
-      acc.y = fmaf(wv[t], ov[t].y, acc.y);
-      acc.z = fmaf(wv[t], ov[t].z, acc.z);
-      acc.w = fmaf(wv[t], ov[t].w, acc.w);
-    }
-  }
   const float gv = p.part[static_cast<int64_t>(slots[0]) * kSlotFloats + QT * BM * D + 2 * QT * BM];
-  const float inv = gv / lsum;
-  const int64_t obase = ((static_cast<int64_t>(b) * p.Lq + qrow) * p.H + h) * D + 4 * lane;
-  if (p.out_bf16) {
-    __nv_bfloat162 v0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    __nv_bfloat162 v1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    uint2 w;
-    w.x = *reinterpret_cast<uint32_t*>(&v0);
-    w.y = *reinterpret_cast<uint32_t*>(&v1);
-    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + obase) = w;
-  } else {
-    *reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase) =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int r = blockIdx.y * kCombineRows + warp * 2 + rr;  // query row of the item
+    const int qrow = m0 + r;
+    if (r >= nq * BM || qrow >= p.Lq) continue;
+    float mstar = -INFINITY, lsum = 0.0f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i0 = 0; i0 < ns; i0 += kCombineParts) {
+      float mv[kCombineParts], lv[kCombineParts];
+      float4 ov[kCombineParts];
+#pragma unroll
+      for (int t = 0; t < kCombineParts; ++t) {  // every load of this group first
+        const int i = i0 + t < ns ? i0 + t : i0;
+        const float* sp = p.part + static_cast<int64_t>(slots[i]) * kSlotFloats;
+        mv[t] = i0 + t < ns ? sp[QT * BM * D + r] : -INFINITY;
+        lv[t] = sp[QT * BM * D + QT * BM + r];
+        ov[t] = reinterpret_cast<const float4*>(sp + r * D)[lane];
+      }
+      float mg = mstar;
+#pragma unroll
+      for (int t = 0; t < kCombineParts; ++t) mg = fmaxf(mg, mv[t]);
+      const float rs = ptx::ex2(mstar - mg);  // 0 while mstar is -inf
+      lsum *= rs;
+      acc = make_float4(acc.x * rs, acc.y * rs, acc.z * rs, acc.w * rs);
+      mstar = mg;
+#pragma unroll
+      for (int t = 0; t < kCombineParts; ++t) {
+        const float wv = i0 + t < ns ? ptx::ex2(mv[t] - mstar) : 0.0f;
+        lsum = fmaf(wv, lv[t], lsum);
+        acc = make_float4(fmaf(wv, ov[t].x, acc.x), fmaf(wv, ov[t].y, acc.y), fmaf(wv, ov[t].z, acc.z),
+                          fmaf(wv, ov[t].w, acc.w));
+      }
+    }
+    const float inv = gv / lsum;
+    const int64_t obase = ((static_cast<int64_t>(b) * p.Lq + qrow) * p.H + h) * D + 4 * lane;
+    if (p.out_bf16) {
+      __nv_bfloat162 v0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      __nv_bfloat162 v1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+      uint2 w;
+      w.x = *reinterpret_cast<uint32_t*>(&v0);
+      w.y = *reinterpret_cast<uint32_t*>(&v1);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + obase) = w;
+    } else {
+      *reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase) =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
   }
 }
 
@@ -1235,7 +1248,7 @@ int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, in
   if (splits) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(prm.pl.G - 1, QT * BM / kCombineRows, 1);
-    cfg.blockDim = dim3(32 * kCombineRows, 1, 1);
+    cfg.blockDim = dim3(32 * kCombineRows / 2, 1, 1);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
