@@ -948,12 +948,12 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
 //   m* = max_k m_k;  O = sum_k O_k 2^(m_k - m*);  l = sum_k l_k 2^(m_k - m*);  out = O g_ref / l
 // (the m_k are whole numbers, so every factor is an exact power of two).  Launched as a
 // programmatic dependent of the attention grid: it waits for that grid before reading partials.
-constexpr int kCombineRows = 16;  // rows of one split item per CTA: 8 warps x 2 rows
+constexpr int kCombineRows = 32;  // rows of one split item per CTA: 8 warps x 4 rows
 constexpr int kCombineParts = 4;  // parts merged with all their loads in flight at once
 
 // One split item's 16 rows: the parts' (m, l, O) rows are all loaded before any is used, so a row
 // costs one round trip to L2 (items split into more than kCombineParts parts loop).
-__global__ void __launch_bounds__(32 * kCombineRows / 2) combine_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(32 * kCombineRows / 4) combine_kernel(const __grid_constant__ AttnParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const Plan& pl = p.pl;
   const int bnd = blockIdx.x + 1;
@@ -993,8 +993,8 @@ __global__ void __launch_bounds__(32 * kCombineRows / 2) combine_kernel(const __
   const int b = bhi / p.H, h = bhi % p.H;
   const float gv = p.part[static_cast<int64_t>(slots[0]) * kSlotFloats + QT * BM * D + 2 * QT * BM];
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int r = blockIdx.y * kCombineRows + warp * 2 + rr;  // query row of the item
+  for (int rr = 0; rr < 4; ++rr) {
+    const int r = blockIdx.y * kCombineRows + warp * 4 + rr;  // query row of the item
     const int qrow = m0 + r;
     if (r >= nq * BM || qrow >= p.Lq) continue;
     float mstar = -INFINITY, lsum = 0.0f;
@@ -1248,7 +1248,7 @@ int launch_attention(const nvfp4kv_cache& c, const uint16_t* q, int q_tokens, in
   if (splits) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(prm.pl.G - 1, QT * BM / kCombineRows, 1);
-    cfg.blockDim = dim3(32 * kCombineRows / 2, 1, 1);
+    cfg.blockDim = dim3(32 * kCombineRows / 4, 1, 1);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
