@@ -507,10 +507,9 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
       float m_run = -INFINITY, l_run = 0.0f;
       // smoothed keys: the logit term scale * log2(e) * q . mu of the (at most two) chunks of the
       // current KV tile, computed when a chunk is first met in this segment
-      int c_lo = -1, c_hi = -1;
+      int c_lo = -1;          // chunk of b_lo; b_hi (when hi_ok) belongs to chunk c_lo + 1
+      bool hi_ok = false;
       float b_lo = 0.0f, b_hi = 0.0f;
-      const float b_factor = p.scale_log2 * q_unscale;
-      const float* const mu_bh = kSmooth ? p.k_mean + bh * p.C * D : nullptr;
       const int nh = 2 * ntl;
       for (int hs = 0; hs < nh && ok; ++hs, ++g) {
         const int jj = jjb + (hs >> 1);
@@ -531,18 +530,18 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         // one cv); any other tile works per column with the same arithmetic.
         const bool uni = info.y != 0;
         // chunk info.z holds columns [0, info.w), chunk info.z + 1 the valid columns after them
-        if (kSmooth && half == 0) {
+        if (kSmooth && half == 0 && (info.z != c_lo || (info.w < BN && !hi_ok))) {
+          // a new chunk: at most two per tile, and the tiles of a segment ascend
+          const float* const mu_bh = p.k_mean + bh * p.C * D;
+          const float f = p.scale_log2 * q_unscale;
           if (info.z != c_lo) {
-            if (info.z == c_hi) {
-              b_lo = b_hi;
-            } else {
-              b_lo = b_factor * q_dot_mean(qrow, row, mu_bh + info.z * D);
-            }
+            b_lo = (hi_ok && info.z == c_lo + 1) ? b_hi : f * q_dot_mean(qrow, row, mu_bh + info.z * D);
             c_lo = info.z;
+            hi_ok = false;
           }
-          if (info.w < BN && info.z + 1 != c_hi) {
-            c_hi = info.z + 1;
-            b_hi = b_factor * q_dot_mean(qrow, row, mu_bh + c_hi * D);
+          if (info.w < BN && !hi_ok) {
+            b_hi = f * q_dot_mean(qrow, row, mu_bh + (c_lo + 1) * D);
+            hi_ok = true;
           }
         }
         const int jsplit = kSmooth ? info.w - half * SUB : 0;  // first column here in chunk info.z + 1
