@@ -35,8 +35,9 @@
 // FP32 scales stay out of the MMAs: g_K(chunk) multiplies S per column, and g_V(chunk) / max g_V
 // multiplies P per column before P is rounded to fp16 (fp16 P and V keep the P V product 8x
 // finer than bf16).  Rows are rescaled lazily: the running max only moves when it grows by more
-// than 2^14 (so P~ stays below 2^14 * 2^(rounding), inside fp16's range).  With smoothed keys (the cache's K-smoothing option) every logit of a chunk's keys
-// also gets scale * q . mu(chunk), computed once per (query row, chunk) from the fp16 Q row.
+// than 2^14 (so P~ stays inside fp16's range).  With smoothed keys (the cache's K-smoothing
+// option) every logit of a chunk's keys also gets scale * q . mu(chunk), computed once per
+// (query row, chunk) from the fp16 Q row.
 //
 // Every mbarrier wait is bounded (%globaltimer); on a time-out the kernel ORs
 // NVFP4KV_ERR_DEVICE_TIMEOUT into the status word, lets in-flight copies and MMAs finish,

@@ -4,7 +4,8 @@
 // (K and V re-quantised to NVFP4 at frame-chunk granularity) and "The NVFP4 quantization
 // format" (FP32 scale, E4M3 scale per 16 elements, E2M1 elements); constants 16 / 448 / 6
 // from the paper page, section 2.2 "NVFP4 Training".  The per-(chunk, head) FP32 scale needs
-// the chunk maximum before any element can be encoded.  Two paths, the same arithmetic:
+// the chunk maximum before any element can be encoded.  Four paths, the same arithmetic (bit-
+// identical codes): for one layer's chunk,
 //   single pass (quantize_cluster_kernel), when one cluster per (b, h, tensor) fits the GPU in
 //       one wave: the cluster's CTAs TMA their token rows into shared memory, reduce max|x|,
 //       exchange the maxima through distributed shared memory, and encode from shared memory
@@ -13,8 +14,11 @@
 //       amax_kernel      every CTA reduces 128 tokens of one (b, h, tensor) to max|x| and writes
 //                        it to a workspace slot (no atomics, no zero-fill, deterministic);
 //       quantize_kernel  launched as a programmatic dependent of the amax grid: every CTA loads
-//                        its 128 rows (from L2, where the first pass just read them), then waits
-//                        for the amax grid, folds the partial maxima into g and encodes.
+//                        its 64 rows (from L2, where the first pass just read them), then waits
+//                        for the amax grid, folds the partial maxima into g and encodes;
+// for the new chunk of many layers at once, quantize_ticket_kernel (one launch, the input read from
+// HBM once; see its own comment); and for caches with the recipe options (K-smoothing, adaptive
+// {4, 6} block scales), key_mean_kernel + recipe_amax_kernel + recipe_encode_kernel.
 // Encoding: two lanes per 16-element block, 16-byte loads, a shuffle for the block maximum,
 // hardware RNE/satfinite conversions to E4M3 and E2M1, 4-byte code stores contiguous across the
 // warp.  Every fp32 step is an explicitly rounded intrinsic (no contraction, no flush to zero),
