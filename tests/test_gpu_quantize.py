@@ -169,3 +169,34 @@ def test_quantize_layers_full_size_equals_per_layer_calls():
     ocache.append(3, *synthetic.chunk_kv(w, 3, 0))
     assert_cache_equal(caches[0], ocache, [3])
     assert caches[0].read_status() == 0
+
+
+def test_quantize_layers_at_the_rollout_step_size():
+    # the benchmark's launch: every one of 30 layers' new 4680-token chunk (12 heads) into slot 39 of
+    # 40-slot caches in one launch; three layers against the oracle, every layer against the
+    # per-layer call
+    import torch
+    w = synthetic.WORKLOADS["rollout"]
+    caches = [KVCache(w.batch, w.heads, w.chunk_tokens, w.capacity) for _ in range(w.layers)]
+    ks, vs = [], []
+    for layer in range(w.layers):
+        k, v = synthetic.device_chunk_kv(w, w.q_chunk, layer)
+        ks.append(k)
+        vs.append(v)
+    quantize_layers(caches, w.q_chunk, ks, vs)
+    assert caches[0].read_status() == 0
+    ref = KVCache(w.batch, w.heads, w.chunk_tokens, w.capacity)
+    t0 = w.q_chunk * w.chunk_tokens
+    for layer in range(w.layers):
+        ref.quantize(w.q_chunk, ks[layer], vs[layer])
+        for name in ("k_codes", "v_codes", "k_scales", "v_scales"):
+            assert torch.equal(getattr(caches[layer], name)[:, :, t0:], getattr(ref, name)[:, :, t0:]), (layer, name)
+        for name in ("k_gscale", "v_gscale"):
+            assert torch.equal(getattr(caches[layer], name)[:, :, w.q_chunk].view(torch.int32),
+                               getattr(ref, name)[:, :, w.q_chunk].view(torch.int32)), (layer, name)
+    for layer in (0, 17, 29):
+        kb = ks[layer].view(torch.int16).cpu().numpy().view(np.uint16)
+        vb = vs[layer].view(torch.int16).cpu().numpy().view(np.uint16)
+        ocache = oracle.Cache(w.batch, w.heads, 128, w.chunk_tokens, w.capacity)
+        ocache.append(w.q_chunk, kb, vb)
+        assert_cache_equal(caches[layer], ocache, [w.q_chunk])
