@@ -109,7 +109,7 @@ def e4m3_encode_array(x: np.ndarray) -> np.ndarray:
 
 def key_mean(x_bf16: np.ndarray, token_stride: int | None = None) -> np.ndarray:
     """K-smoothing's channel mean of one chunk ``x_bf16`` (uint16 [B, L, H, d]): float32 [B, H, d],
-    the fp32 rounding of the fp64 token-order sum divided by L."""
+    the exact mean rounded once to fp32 (nearest, ties to even)."""
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
     B, L, H, d = x.shape
     stride = H * d if token_stride is None else token_stride

@@ -27,8 +27,9 @@
  *  The pages' own recipe for the cache [N2]: "K-smoothing" of K and "adaptive scale selection"
  *  of V within each chunk, with the candidate scale targets {4, 6} [N3], [P1 sec. A.2].  The
  *  pages name both and define neither; the readings taken here:
- *   K-smoothing: mu_i = (float)((sum over t of x[t][i], in fp64, t = 0, 1, ... in order) / L),
- *     the channel mean of the chunk's keys of one head; the chunk is quantised as above from
+ *   K-smoothing: mu_i = the channel mean of the chunk's keys of one head, (sum over t of x[t][i]) / L
+ *     computed exactly (every bf16 value is a whole number of 2^-133) and rounded once to fp32,
+ *     to nearest with ties to even; the chunk is quantised as above from
  *     x'[t][i] = x[t][i] - mu_i (one fp32 subtraction), and the key the cache stands for is
  *     x_hat' + mu (mu stored in fp32 beside the chunk).
  *   Adaptive scale (target T in {6, 4}): for every block both targets are tried,
@@ -44,6 +45,7 @@
  */
 #include "nvfp4kv_oracle.h"
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <limits>
@@ -64,6 +66,94 @@ float bf16_bits_to_float(uint16_t h) {
   float f;
   std::memcpy(&f, &u, sizeof f);
   return f;
+}
+
+/* A non-negative integer as little-endian 32-bit digits: just enough arithmetic for the exact
+ * channel mean (add a small value shifted left, compare, subtract, divide by a small value). */
+struct BigNat {
+  std::vector<uint32_t> dig;
+  void add_shifted(uint32_t m, int shift) {
+    size_t k = static_cast<size_t>(shift / 32);
+    uint64_t carry = static_cast<uint64_t>(m) << (shift % 32);
+    while (carry != 0) {
+      if (dig.size() <= k) dig.resize(k + 1, 0u);
+      const uint64_t t = static_cast<uint64_t>(dig[k]) + (carry & 0xFFFFFFFFu);
+      dig[k] = static_cast<uint32_t>(t);
+      carry = (carry >> 32) + (t >> 32);
+      ++k;
+    }
+  }
+  bool bit(int n) const {
+    const size_t k = static_cast<size_t>(n / 32);
+    return k < dig.size() && ((dig[k] >> (n % 32)) & 1u);
+  }
+  int bit_length() const {
+    for (size_t k = dig.size(); k-- > 0;)
+      if (dig[k] != 0)
+        for (int j = 31; j >= 0; --j)
+          if ((dig[k] >> j) & 1u) return static_cast<int>(k) * 32 + j + 1;
+    return 0;
+  }
+};
+
+int compare(const BigNat& a, const BigNat& b) {
+  const size_t n = std::max(a.dig.size(), b.dig.size());
+  for (size_t k = n; k-- > 0;) {
+    const uint32_t x = k < a.dig.size() ? a.dig[k] : 0u, y = k < b.dig.size() ? b.dig[k] : 0u;
+    if (x != y) return x < y ? -1 : 1;
+  }
+  return 0;
+}
+
+BigNat subtract(const BigNat& a, const BigNat& b) { /* a >= b */
+  BigNat r;
+  r.dig.resize(a.dig.size(), 0u);
+  int64_t borrow = 0;
+  for (size_t k = 0; k < a.dig.size(); ++k) {
+    int64_t t = static_cast<int64_t>(a.dig[k]) - (k < b.dig.size() ? b.dig[k] : 0u) - borrow;
+    borrow = t < 0 ? 1 : 0;
+    if (t < 0) t += (int64_t(1) << 32);
+    r.dig[k] = static_cast<uint32_t>(t);
+  }
+  return r;
+}
+
+/* fp32 nearest to (pos - neg) * 2^-133 / L, ties to even: the quotient is taken in units of 2^-149
+ * (the smallest fp32 subnormal step) with its remainder, then rounded to 24 significant bits. */
+float exact_mean_to_float(const BigNat& pos, const BigNat& neg, uint32_t L) {
+  const int c = compare(pos, neg);
+  if (c == 0) return 0.0f;
+  BigNat mag = c > 0 ? subtract(pos, neg) : subtract(neg, pos);
+  BigNat num;  /* mag * 2^16 */
+  for (int n = mag.bit_length() - 1; n >= 0; --n)
+    if (mag.bit(n)) num.add_shifted(1u, n + 16);
+  /* long division by L, most significant digit first */
+  BigNat q;
+  q.dig.resize(num.dig.size(), 0u);
+  uint64_t r = 0;
+  for (size_t k = num.dig.size(); k-- > 0;) {
+    const uint64_t cur = (r << 32) | num.dig[k];
+    q.dig[k] = static_cast<uint32_t>(cur / L);
+    r = cur % L;
+  }
+  const int n = q.bit_length();
+  double v;
+  if (n <= 24) { /* below 2^-125: every multiple of 2^-149 under 2^24 of them is an fp32 value */
+    uint64_t k = 0;
+    for (int j = n - 1; j >= 0; --j) k = (k << 1) | (q.bit(j) ? 1u : 0u);
+    const bool up = 2 * r > L || (2 * r == L && (k & 1u));
+    v = std::ldexp(static_cast<double>(k + (up ? 1 : 0)), -149);
+  } else {
+    const int sh = n - 24;
+    uint64_t mant = 0;
+    for (int j = n - 1; j >= sh; --j) mant = (mant << 1) | (q.bit(j) ? 1u : 0u);
+    const bool guard = q.bit(sh - 1);
+    bool lower = r != 0;
+    for (int j = sh - 2; j >= 0 && !lower; --j) lower = q.bit(j);
+    const bool up = guard && (lower || (mant & 1u));
+    v = std::ldexp(static_cast<double>(mant + (up ? 1 : 0)), sh - 149);
+  }
+  return static_cast<float>(c > 0 ? v : -v); /* exact: v has at most 24 significant bits */
 }
 
 /* Nearest code among the ascending non-negative magnitudes dec(0) < dec(1) < ... <
@@ -138,17 +228,24 @@ void oracle_e4m3_encode_array(const float* x, int64_t n, uint8_t* out) {
 
 int oracle_key_mean(const uint16_t* x, int32_t B, int32_t L, int32_t H, int32_t d,
                     int64_t token_stride, float* mean) {
-  if (!x || !mean || B <= 0 || L <= 0 || H <= 0 || d <= 0 || token_stride < static_cast<int64_t>(H) * d)
+  if (!x || !mean || B <= 0 || L <= 0 || L > (1 << 23) || H <= 0 || d <= 0 ||
+      token_stride < static_cast<int64_t>(H) * d)
     return -1;
-  IeeeMode ieee;
   for (int32_t b = 0; b < B; ++b)
     for (int32_t h = 0; h < H; ++h)
       for (int32_t i = 0; i < d; ++i) {
-        double sum = 0.0;
-        for (int32_t t = 0; t < L; ++t)  /* token order */
-          sum += static_cast<double>(bf16_bits_to_float(
-              x[(static_cast<int64_t>(b) * L + t) * token_stride + static_cast<int64_t>(h) * d + i]));
-        mean[(static_cast<int64_t>(b) * H + h) * d + i] = static_cast<float>(sum / L);
+        /* the exact sum of the channel, as counts of 2^-133 (every bf16 value is a whole number of
+         * them): positive and negative values kept apart, each a non-negative big integer */
+        BigNat pos, neg;
+        for (int32_t t = 0; t < L; ++t) {
+          const uint16_t v = x[(static_cast<int64_t>(b) * L + t) * token_stride + static_cast<int64_t>(h) * d + i];
+          const int e = (v >> 7) & 0xFF, f = v & 0x7F;
+          /* |v| = f * 2^-133 (e == 0), else (128 + f) * 2^(e - 134) = ((128 + f) << (e - 1)) * 2^-133 */
+          const uint32_t m = e == 0 ? static_cast<uint32_t>(f) : static_cast<uint32_t>(128 + f);
+          const int shift = e == 0 ? 0 : e - 1;
+          ((v & 0x8000) ? neg : pos).add_shifted(m, shift);
+        }
+        mean[(static_cast<int64_t>(b) * H + h) * d + i] = exact_mean_to_float(pos, neg, static_cast<uint32_t>(L));
       }
   return 0;
 }

@@ -60,8 +60,9 @@ void oracle_e4m3_encode_array(const float* x, int64_t n, uint8_t* out);
 int oracle_quantize_chunk(const uint16_t* x, int32_t B, int32_t L, int32_t H, int32_t d,
                           int64_t token_stride, uint8_t* codes, uint8_t* scales, float* gscale);
 
-/* K-smoothing [N2]: the channel mean of one chunk's keys per (b, h), as the fp32 rounding of the
- * fp64 sum over the chunk's tokens in token order divided by L.  mean: [B][H][d].  Returns 0 / -1. */
+/* K-smoothing [N2]: the channel mean of one chunk's keys per (b, h): the exact sum over the chunk's
+ * L tokens divided by L, rounded once to fp32 (nearest, ties to even).  mean: [B][H][d].
+ * Returns 0, or -1 for bad sizes (L above 2^23 included). */
 int oracle_key_mean(const uint16_t* x, int32_t B, int32_t L, int32_t H, int32_t d,
                     int64_t token_stride, float* mean);
 

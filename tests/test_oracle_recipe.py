@@ -3,8 +3,8 @@ infrastructure": K-smoothing of K and adaptive scale selection of V within each 
 note, "Engineering details of NVFP4 training": candidate scale magnitudes {4, 6}).
 
 The pages name both options and define neither.  The readings pinned here:
-  K-smoothing  mu = fp32(fp64 token-order sum / L) per channel; x - mu is quantised; the key the
-               cache stands for is x_hat' + mu.
+  K-smoothing  mu = the exact channel mean rounded once to fp32 (nearest, ties to even); x - mu
+               is quantised; the key the cache stands for is x_hat' + mu.
   adaptive     per 16-element block, scale targets 6 and 4 are both tried and the one with the
                smaller fp64 squared error kept (ties keep 6); g is unchanged.
 Each expected value below follows from the format constants by hand, from a closed form, or from
@@ -60,12 +60,69 @@ def test_key_mean_of_constant_and_arithmetic_channels():
     assert mu[0, 0, 9] == 0.0
 
 
-def test_key_mean_sums_in_token_order():
-    # 2^60 + 1 rounds back to 2^60 in fp64, so the token-order sum of [2^60, 1, -2^60, 1] is 1
-    # and the mean 0.25 (the exact mean is 0.5; a pairwise sum would give 0)
+def test_key_mean_is_exact_whatever_the_order():
+    # [2^60, 1, -2^60, 1]: an fp64 running sum would lose the first 1 (2^60 + 1 rounds back to
+    # 2^60) and give 0.25, a pairwise one 0; the exact mean is 0.5
     x = np.zeros((1, 4, 1, 16))
     x[0, :, 0, 0] = [2.0 ** 60, 1.0, -(2.0 ** 60), 1.0]
-    assert oracle.key_mean(_bits(x))[0, 0, 0] == np.float32(0.25)
+    x[0, :, 0, 1] = [1.0, 2.0 ** 60, 1.0, -(2.0 ** 60)]
+    mu = oracle.key_mean(_bits(x))
+    assert mu[0, 0, 0] == np.float32(0.5) and mu[0, 0, 1] == np.float32(0.5)
+
+
+def test_key_mean_rounds_once_to_nearest_even():
+    # (2^24 + 1) / 2 = 2^23 + 0.5 and (2^24 + 3) / 2 = 2^23 + 1.5 are exact fp32 midpoints: ties go
+    # to the even significand; (2^24 + 2^17 + 1 + 2^-7) / 2 lies just above a midpoint and rounds up
+    x = np.zeros((1, 2, 1, 16))
+    x[0, :, 0, 0] = [2.0 ** 24, 1.0]
+    x[0, :, 0, 1] = [2.0 ** 24, 3.0]
+    x[0, :, 0, 2] = [2.0 ** 24 + 2.0 ** 17, 1.0 + 2.0 ** -7]  # mean 2^23 + 2^16 + 0.5 + 2^-8
+    x[0, :, 0, 3] = [-(2.0 ** 24), -1.0]
+    mu = oracle.key_mean(_bits(x))
+    assert mu[0, 0, 0] == np.float32(2.0 ** 23)
+    assert mu[0, 0, 1] == np.float32(2.0 ** 23 + 2.0)
+    assert mu[0, 0, 2] == np.float32(2.0 ** 23 + 2.0 ** 16 + 1.0)
+    assert mu[0, 0, 3] == np.float32(-(2.0 ** 23))
+
+
+def _fp32_nearest(q):
+    """Nearest fp32 to the rational q, ties to even, by bisection over positive bit patterns."""
+    from fractions import Fraction
+    import struct
+    if q == 0:
+        return 0.0
+    neg, a = q < 0, abs(q)
+    val = lambda u: Fraction(struct.unpack("<f", struct.pack("<I", u))[0])
+    lo, hi = 0, 0x7F7FFFFF  # largest pattern with value <= a
+    while lo < hi:
+        mid = (lo + hi + 1) // 2
+        if val(mid) <= a:
+            lo = mid
+        else:
+            hi = mid - 1
+    below, above = val(lo), val(lo + 1)
+    pick = lo if (a - below < above - a or (a - below == above - a and lo % 2 == 0)) else lo + 1
+    f = struct.unpack("<f", struct.pack("<I", pick))[0]
+    return -f if neg else f
+
+
+def test_key_mean_against_exact_rationals():
+    from fractions import Fraction
+    rng = np.random.default_rng(21)
+    for L, scale in ((3, 1.0), (7, 2.0 ** -130), (64, 2.0 ** 100), (200, 1.0), (5, 2.0 ** -140)):
+        v = rng.standard_normal((1, L, 1, 16)) * scale * np.exp2(rng.integers(-20, 21, size=(1, L, 1, 16)))
+        bits = _bits(v, exact=False)
+        mu = oracle.key_mean(bits)
+        vals = _val(bits)
+        for i in range(16):
+            want = _fp32_nearest(sum(Fraction(float(t)) for t in vals[0, :, 0, i]) / L)
+            assert mu[0, 0, i] == np.float32(want), (L, scale, i)
+    # a lone smallest subnormal among zeros: 2^-133 / 3 lies between fp32 subnormals
+    x = np.zeros((1, 3, 1, 16))
+    x[0, 0, 0, 0] = 2.0 ** -133
+    mu = oracle.key_mean(_bits(x))
+    assert mu[0, 0, 0] == np.float32(_fp32_nearest(Fraction(2) ** -133 / 3))
+    assert mu[0, 0, 0] == np.float32(21845 * 2.0 ** -149)  # 2^16 / 3 = 21845.33 steps of 2^-149
 
 
 def test_key_mean_per_head_and_batch_with_token_stride():
