@@ -32,7 +32,9 @@
  * section A.2, cites adaptive block-scale selection ("Four Over Six") for lower NVFP4 error.  The
  * pages define neither; this library reads them as:
  *  NVFP4KV_K_SMOOTH: per (chunk, head) the channel mean of the chunk's keys,
- *      mu_e = fp32( (sum over t = 0, 1, ... of x[t][e], in fp64 in token order) / chunk_tokens ),
+ *      mu_e = (sum over t of x[t][e]) / chunk_tokens, computed exactly and rounded once to fp32
+ *      (nearest, ties to even; a key with an Inf or NaN bit pattern counts as the finite number
+ *      (1 + f / 128) * 2^128 of its fraction bits f),
  *    is stored in k_mean and the chunk is quantised as above from x' = x - mu (one fp32
  *    subtraction per element); the key the cache holds is x_hat' + mu, and attention adds the
  *    per-(query row, chunk) term q . mu to every logit of the chunk's keys.
@@ -84,8 +86,9 @@ typedef enum { NVFP4KV_OUT_F32 = 0, NVFP4KV_OUT_BF16 = 1 } nvfp4kv_out_dtype;
  *   status             uint32, one word; zero it once before first use
  *   k_mean             fp32  [batch][heads][capacity_chunks][head_dim] (NVFP4KV_K_SMOOTH only)
  * Every array must start on a 16-byte boundary.  flags with bits other than the two options,
- * or NVFP4KV_K_SMOOTH without k_mean, is NVFP4KV_ERR_INVALID_ARG for every call; one cache keeps
- * its flags for its whole life (its slots are read as they were written). */
+ * or NVFP4KV_K_SMOOTH without k_mean, is NVFP4KV_ERR_INVALID_ARG for every call, and
+ * NVFP4KV_K_SMOOTH with chunk_tokens > 2^23 is NVFP4KV_ERR_UNSUPPORTED for every call; one cache
+ * keeps its flags for its whole life (its slots are read as they were written). */
 typedef struct {
   int32_t batch;
   int32_t heads;

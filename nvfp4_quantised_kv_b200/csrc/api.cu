@@ -33,6 +33,8 @@ int check_cache(const nvfp4kv_cache* c) {
   if (reinterpret_cast<uintptr_t>(c->status) & 3u) return NVFP4KV_ERR_INVALID_ARG;
   if (c->flags & ~static_cast<uint32_t>(NVFP4KV_K_SMOOTH | NVFP4KV_V_ADAPTIVE_SCALE)) return NVFP4KV_ERR_INVALID_ARG;
   if ((c->flags & NVFP4KV_K_SMOOTH) && (!c->k_mean || !aligned16(c->k_mean))) return NVFP4KV_ERR_INVALID_ARG;
+  // the channel-mean kernel's exact integer sums have headroom for 2^23 keys per chunk
+  if ((c->flags & NVFP4KV_K_SMOOTH) && c->chunk_tokens > (1 << 23)) return NVFP4KV_ERR_UNSUPPORTED;
   return NVFP4KV_OK;
 }
 

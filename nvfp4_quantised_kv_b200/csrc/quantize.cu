@@ -239,10 +239,10 @@ __global__ void __launch_bounds__(kThreads, 6) quantize_kernel(const __grid_cons
 // block-scale targets of V (reading note, "The inference infrastructure": both applied within
 // each chunk; "Engineering details of NVFP4 training": candidate scale magnitudes {4, 6}).
 //   key_mean_kernel       one CTA per (32 channels, b, h): TMA brings 64-token slices of the
-//                         chunk's keys into a ring in shared memory and one warp adds them up, a
-//                         lane per channel, in fp64 in token order; mu = fp32(sum / L) is written
-//                         to the slot's k_mean.  (The sum is one dependent chain per channel:
-//                         its order is part of the definition.)
+//                         chunk's keys into a ring in shared memory; eight warps add them, a lane
+//                         per channel, exactly (an fp64 sum per slice where that is exact, integer
+//                         bins otherwise), and the exact mean rounded once to fp32 is written to
+//                         the slot's k_mean.
 //   recipe_amax_kernel    amax_kernel over x - mu for a smoothed K (fp32 magnitudes); the
 //                         partials hold fp32 bit patterns for both tensors.
 //   recipe_encode_kernel  quantize_kernel from x - mu for a smoothed K; for V with adaptive
@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 6) quantize_kernel(const __grid_cons
 //                         with the smaller fp64 squared error, ties keeping 6.
 constexpr int kMeanTok = 64;    // tokens per ring stage
 constexpr int kMeanCh = 32;     // channels per CTA (64 bytes of each token row)
-constexpr int kMeanStages = 8;  // 8 x 4 KB in flight per CTA
+constexpr int kMeanStages = 16;  // 16 x 4 KB in flight per CTA
 
 struct MeanArgs {
   float* k_mean;
@@ -269,27 +269,117 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-__global__ void __launch_bounds__(64) key_mean_kernel(const __grid_constant__ CUtensorMap tm,
-                                                      const __grid_constant__ MeanArgs a) {
-  __shared__ __align__(128) uint16_t ring[kMeanStages][kMeanTok * kMeanCh];
+// fp32 nearest (ties to even) to S * 2^-133 / L for the exact signed integer S given as 32-bit
+// digits d[0..n) (two's complement, d[n-1] holding the sign): the mean of L bf16 values whose
+// sum is S units of 2^-133.  The magnitude is shifted into units of 2^-149 (the fp32 subnormal
+// step), divided by L with its remainder, and rounded to 24 significant bits.
+template <int n>
+__device__ float exact_mean_to_f32(uint32_t (&d)[n], uint32_t L) {
+  const bool neg = (d[n - 1] >> 31) != 0u;
+  if (neg) {  // magnitude: two's complement negation
+    uint32_t carry = 1u;
+#pragma unroll
+    for (int k = 0; k < n; ++k) {
+      const uint64_t t = static_cast<uint64_t>(~d[k]) + carry;
+      d[k] = static_cast<uint32_t>(t);
+      carry = static_cast<uint32_t>(t >> 32);
+    }
+  }
+  // times 2^16: units of 2^-149 (the top digit has room: |S| < 2^285 for L <= 2^23)
+#pragma unroll
+  for (int k = n - 1; k > 0; --k) d[k] = (d[k] << 16) | (d[k - 1] >> 16);
+  d[0] <<= 16;
+  // divided by L, most significant digit first
+  uint64_t r = 0;
+#pragma unroll
+  for (int k = n - 1; k >= 0; --k) {
+    const uint64_t cur = (r << 32) | d[k];
+    d[k] = static_cast<uint32_t>(cur / L);
+    r = cur % L;
+  }
+  int top = -1;  // highest non-zero digit of the quotient
+#pragma unroll
+  for (int k = 0; k < n; ++k)
+    if (d[k] != 0u) top = k;
+  if (top < 0 && r == 0) return 0.0f;
+  const int nbits = top < 0 ? 0 : top * 32 + (32 - __clz(d[top]));  // bit length of the quotient
+  auto bit = [&](int j) -> uint32_t {  // bit j of the quotient (j >= 0)
+    uint32_t v = 0u;
+#pragma unroll
+    for (int k = 0; k < n; ++k)
+      if (k == (j >> 5)) v = (d[k] >> (j & 31)) & 1u;
+    return v;
+  };
+  double v;
+  if (nbits <= 24) {  // below 2^-125: every whole number of 2^-149 up to 2^24 is an fp32 value
+    const uint64_t q = (top < 0) ? 0u : (top == 0 ? d[0] : (static_cast<uint64_t>(d[1]) << 32) | d[0]);
+    const bool up = 2 * r > L || (2 * r == L && (q & 1u));
+    v = ldexp(static_cast<double>(q + (up ? 1u : 0u)), -149);
+  } else {
+    const int sh = nbits - 24;
+    uint64_t mant = 0;
+    for (int j = nbits - 1; j >= sh; --j) mant = (mant << 1) | bit(j);
+    const bool guard = bit(sh - 1) != 0u;
+    bool lower = r != 0;
+    for (int j = sh - 2; j >= 0 && !lower; --j) lower = bit(j) != 0u;
+    const bool up = guard && (lower || (mant & 1u));
+    v = ldexp(static_cast<double>(mant + (up ? 1u : 0u)), sh - 149);
+  }
+  return __double2float_rn(neg ? -v : v);  // exact: at most 24 significant bits
+}
+
+// K-smoothing's channel means of one chunk: the exact mean of each channel's L bf16 keys, rounded
+// once to fp32.  Every bf16 value is a whole number of 2^-133 (< 2^261 of them), so the sum is
+// kept exactly as integers in nine 64-bit bins per channel, bin k counting units of 2^(32 k - 133):
+// integer additions, so any order gives the same sum and the tokens are summed in parallel.
+// One CTA per (32 channels, b, h): a producer lane TMA-loads 64-token x 32-channel boxes into a
+// 16-stage ring; eight warps take the stages in turn, a lane per channel, each thread adding into
+// bins of its own, which are summed at the end.
+// A lane first sums its 64 values of a stage in fp64.  When the stage's non-zero magnitudes span
+// at most 40 binades (2^(pos_hi - pos_lo) <= 2^39) every partial sum is a whole number of
+// 2^(pos_lo - 133) below 2^(8 + 39 + 6) = 2^53, so fp64 holds each one exactly, in any order; the
+// exact stage sum then goes into three bins as 32-bit pieces.  Other stages (a wider span, or an
+// Inf/NaN bit pattern, which the bins read as the number its bits spell) are added value by value
+// into the bins instead.  Each bin stays below 2^63 in magnitude for L <= 2^23: at most L values
+// below 2^39 each, plus one piece below 2^32 per stage.
+constexpr int kMeanWarps = 8;   // consumer warps
+constexpr int kMeanBins = 9;    // a value lands in bin (pos >> 5) <= 7, a stage sum in bins <= 8
+constexpr int kMeanSpan = 39;   // widest exponent span a stage may have for its fp64 sum
+constexpr size_t kMeanSmem = static_cast<size_t>(kMeanStages) * kMeanTok * kMeanCh * 2;  // the ring
+
+// |v| = m * 2^(pos - 133) for the bf16 bit pattern v: m < 256, 0 <= pos <= 254
+__device__ __forceinline__ void bf16_units(uint32_t v, uint32_t& m, uint32_t& pos) {
+  const uint32_t e = (v >> 7) & 0xFFu, f = v & 0x7Fu;
+  m = e == 0u ? f : 128u + f;
+  pos = e == 0u ? 0u : e - 1u;
+}
+
+__global__ void __launch_bounds__(32 * (kMeanWarps + 1)) key_mean_kernel(const __grid_constant__ CUtensorMap tm,
+                                                                         const __grid_constant__ MeanArgs a) {
+  extern __shared__ __align__(128) uint16_t ring[];  // [kMeanStages][kMeanTok][kMeanCh]
   __shared__ __align__(8) uint64_t full[kMeanStages], empty[kMeanStages];
+  __shared__ unsigned long long bins[kMeanWarps][kMeanBins][kMeanCh];  // each slot owned by one thread
   __shared__ int s_issued;
+  __shared__ int s_bad;
   const int cg = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = (a.L + kMeanTok - 1) / kMeanTok;
+  for (int i = threadIdx.x; i < kMeanWarps * kMeanBins * kMeanCh; i += blockDim.x) (&bins[0][0][0])[i] = 0ull;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMeanStages; ++i) {
       ptx::mbar_init(ptx::smem_u32(&full[i]), 1);
       ptx::mbar_init(ptx::smem_u32(&empty[i]), 1);
     }
     ptx::fence_mbar_init();
+    s_issued = 0;
+    s_bad = 0;
   }
   __syncthreads();
   bool ok = true;
-  if (warp == 1) {
-    // producer: one TMA box (64 tokens x 32 channels) per stage; a stage is reused once the
-    // summing warp has released it
+  if (warp == kMeanWarps) {
+    // producer: one TMA box (64 tokens x 32 channels) per stage; a stage is reused once the warp
+    // that summed it has released it
     if (lane == 0) {
       int issued = 0;
       for (int i = 0; i < n_tiles; ++i) {
@@ -299,42 +389,114 @@ __global__ void __launch_bounds__(64) key_mean_kernel(const __grid_constant__ CU
           break;
         }
         ptx::mbar_arrive_expect_tx(ptx::smem_u32(&full[st]), kMeanTok * kMeanCh * 2);
-        ptx::tma_load_4d(ptx::smem_u32(ring[st]), &tm, cg * kMeanCh, h, i * kMeanTok, b, ptx::smem_u32(&full[st]));
+        ptx::tma_load_4d(ptx::smem_u32(ring + st * kMeanTok * kMeanCh), &tm, cg * kMeanCh, h, i * kMeanTok, b,
+                         ptx::smem_u32(&full[st]));
         ++issued;
       }
       s_issued = issued;
     }
   } else {
-    // one lane per channel: the fp64 sum in token order
-    double sum = 0.0;
-    for (int i = 0; i < n_tiles; ++i) {
+    // warp w sums the stages of tiles w, w + 8, ...; lane = channel
+    unsigned long long* my = &bins[warp][0][lane];  // bin k of this thread: my[k * kMeanCh]
+    for (int i = warp; i < n_tiles; i += kMeanWarps) {
       const int st = i % kMeanStages;
       ok = __all_sync(0xFFFFFFFFu, wait_phase(ptx::smem_u32(&full[st]), (i / kMeanStages) & 1));
       if (!ok) break;
       const int n = min(kMeanTok, a.L - i * kMeanTok);
-      const uint16_t* col = ring[st] + lane;
+      const uint16_t* col = ring + st * kMeanTok * kMeanCh + lane;
+      // fp64 sum of the stage, with the largest magnitude and the smallest non-zero one (as bit
+      // patterns: a zero's pattern less one wraps to the top and never wins the minimum)
+      double s[4] = {0.0, 0.0, 0.0, 0.0};
+      uint32_t hi = 0u, lo_m1 = 0xFFFFFFFFu;
       if (n == kMeanTok) {
-        // a full stage: every shared-memory load first, then the dependent adds in token order
-        uint16_t v[kMeanTok];
-        const uint32_t base = ptx::smem_u32(col);
+        uint32_t v[kMeanTok];
 #pragma unroll
-        for (int t = 0; t < kMeanTok; ++t)  // volatile: all 64 loads stay ahead of the adds
-          asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v[t]) : "r"(base + t * kMeanCh * 2));
+        for (int t = 0; t < kMeanTok; ++t) v[t] = col[t * kMeanCh];
 #pragma unroll
-        for (int t = 0; t < kMeanTok; ++t) sum += static_cast<double>(__uint_as_float(static_cast<uint32_t>(v[t]) << 16));
+        for (int t = 0; t < kMeanTok; ++t) {
+          const uint32_t mag = v[t] & 0x7FFFu;
+          hi = max(hi, mag);
+          lo_m1 = min(lo_m1, mag - 1u);
+          s[t & 3] = __dadd_rn(s[t & 3], static_cast<double>(__uint_as_float(v[t] << 16)));
+        }
       } else {
-        for (int t = 0; t < n; ++t) sum += static_cast<double>(__uint_as_float(static_cast<uint32_t>(col[t * kMeanCh]) << 16));
+        for (int t = 0; t < n; ++t) {
+          const uint32_t v = col[t * kMeanCh];
+          const uint32_t mag = v & 0x7FFFu;
+          hi = max(hi, mag);
+          lo_m1 = min(lo_m1, mag - 1u);
+          s[0] = __dadd_rn(s[0], static_cast<double>(__uint_as_float(v << 16)));
+        }
+      }
+      bool exact = hi < 0x7F80u;  // finite
+      if (exact && hi != 0u) {
+        const uint32_t lo = lo_m1 + 1u;
+        const int p_hi = hi >= 0x80u ? static_cast<int>(hi >> 7) - 1 : 0;
+        const int p_lo = lo >= 0x80u ? static_cast<int>(lo >> 7) - 1 : 0;
+        exact = p_hi - p_lo <= kMeanSpan;
+      }
+      if (exact) {
+        const double sum = __dadd_rn(__dadd_rn(s[0], s[1]), __dadd_rn(s[2], s[3]));
+        if (sum != 0.0) {
+          // sum = M * 2^(E - 1075) = M * 2^sh units of 2^-133; a whole number of them, so a
+          // negative sh only drops zero bits of M
+          const unsigned long long sb = static_cast<unsigned long long>(__double_as_longlong(sum));
+          unsigned long long M = (sb & 0xFFFFFFFFFFFFFull) | (1ull << 52);
+          int sh = static_cast<int>((sb >> 52) & 0x7FFu) - 942;
+          if (sh < 0) {
+            M >>= -sh;
+            sh = 0;
+          }
+          const int k = sh >> 5, r = sh & 31;  // |sum| < 2^267 units: sh <= 214, k + 2 <= 8
+          const unsigned long long lo64 = M << r, hi64 = r ? M >> (64 - r) : 0ull;
+          unsigned long long p0 = lo64 & 0xFFFFFFFFull, p1 = lo64 >> 32, p2 = hi64;
+          if (sb >> 63) {
+            p0 = 0ull - p0;
+            p1 = 0ull - p1;
+            p2 = 0ull - p2;
+          }
+          my[k * kMeanCh] += p0;
+          my[(k + 1) * kMeanCh] += p1;
+          my[(k + 2) * kMeanCh] += p2;
+        }
+      } else {
+        // value by value: bin (pos >> 5) gets m * 2^(pos & 31), negated for a negative value
+        for (int t = 0; t < n; ++t) {
+          const uint32_t v = col[t * kMeanCh];
+          if ((v & 0x7FFFu) == 0u) continue;  // +-0 adds nothing
+          uint32_t m, pos;
+          bf16_units(v, m, pos);
+          unsigned long long add = static_cast<unsigned long long>(m) << (pos & 31u);
+          if (v & 0x8000u) add = 0ull - add;  // two's complement: the bins wrap, the sums do not
+          my[(pos >> 5) * kMeanCh] += add;
+        }
       }
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty[st]));
     }
-    if (ok)
-      a.k_mean[(static_cast<int64_t>(bh) * a.C + a.slot) * kHeadDim + cg * kMeanCh + lane] =
-          __double2float_rn(sum / static_cast<double>(a.L));
+    if (!ok && lane == 0) atomicOr(&s_bad, 1);
   }
-  if (!ok && (lane == 0)) atomicOr(a.status, kStatusTimeout);
+  if (!ok && lane == 0) atomicOr(a.status, kStatusTimeout);
   __syncthreads();
-  if (threadIdx.x == 32) {
+  if (warp == 0 && s_bad == 0 && s_issued == n_tiles) {
+    // S = sum over bins of bins[k] * 2^(32 k) as 32-bit digits (two's complement), then the mean
+    constexpr int kDigits = kMeanBins + 1;
+    uint32_t d[kDigits];
+    int64_t carry = 0;
+#pragma unroll
+    for (int k = 0; k < kDigits; ++k) {
+      unsigned long long bk = 0ull;  // bin k of this channel over the warps (wrapping sum)
+      if (k < kMeanBins)
+#pragma unroll
+        for (int w = 0; w < kMeanWarps; ++w) bk += bins[w][k][lane];
+      const int64_t acc = carry + static_cast<int64_t>(bk);
+      d[k] = static_cast<uint32_t>(acc);           // the low 32 bits
+      carry = (acc - static_cast<int64_t>(d[k])) / (int64_t(1) << 32);  // exact: the rest is a multiple
+    }
+    a.k_mean[(static_cast<int64_t>(bh) * a.C + a.slot) * kHeadDim + cg * kMeanCh + lane] =
+        exact_mean_to_f32<kDigits>(d, static_cast<uint32_t>(a.L));
+  }
+  if (threadIdx.x == 32 * kMeanWarps) {
     // after a time-out some copies may still be in flight: let them land (bounded) before the
     // CTA's shared memory goes away
     for (int i = max(0, s_issued - kMeanStages); i < s_issued; ++i)
@@ -996,6 +1158,8 @@ cudaError_t launch_encode_dependent(Kernel kernel, const QuantArgs& a, cudaStrea
   return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
+PerDeviceOnce g_mean_attr;
+
 cudaError_t launch_quantize_recipe(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
                                    int64_t token_stride, void* workspace, cudaStream_t stream) {
   const QuantArgs a = two_pass_args(c, slot, k, v, token_stride, workspace);
@@ -1020,7 +1184,12 @@ cudaError_t launch_quantize_recipe(const nvfp4kv_cache& c, int slot, const uint1
     m.L = c.chunk_tokens;
     m.C = c.capacity_chunks;
     m.slot = slot;
-    key_mean_kernel<<<dim3(kHeadDim / kMeanCh, c.batch * c.heads), 64, 0, stream>>>(tm, m);
+    const cudaError_t attr_err = g_mean_attr.run([] {
+      return cudaFuncSetAttribute(key_mean_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kMeanSmem));
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    key_mean_kernel<<<dim3(kHeadDim / kMeanCh, c.batch * c.heads), 32 * (kMeanWarps + 1), kMeanSmem, stream>>>(tm, m);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

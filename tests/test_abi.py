@@ -181,6 +181,10 @@ def test_recipe_flags_are_checked_before_any_launch(L):
                               1 << 24, None)
     assert rc == nk.ERR_UNSUPPORTED
     del out
+    # smoothed chunks beyond 2^23 keys: more than the exact channel sums have room for
+    long_chunk = _desc(flags=nk.K_SMOOTH, k_mean=0xB0000, chunk_tokens=(1 << 23) + 2, capacity_chunks=1)
+    assert _quant(L, long_chunk) == nk.ERR_UNSUPPORTED
+    assert L.nvfp4_kv_dequantize(ctypes.byref(long_chunk), 0, 0, 1, 0x90000, None) == nk.ERR_UNSUPPORTED
     # the single-launch multi-layer quantiser takes plain caches only
     pair = (nk.CacheDesc * 2)(_desc(), _desc(flags=nk.V_ADAPTIVE_SCALE))
     ks = (ctypes.c_void_p * 2)(0x80000, 0x80000)

@@ -97,6 +97,51 @@ def test_recipe_token_stride_and_ragged_length():
     _assert_means_equal(cache, ocache, [1])
 
 
+def _adversarial_keys(B, L, H, seed):
+    """Keys whose channels stress an exact sum: eight kinds, by channel mod 8 (uint16 [B, L, H, 128])."""
+    rng = np.random.default_rng(seed)
+    x = f32_to_bf16_bits((rng.standard_normal((B, L, H, 128)) * 3.0 + 1.0).astype(np.float32))
+    sign = lambda n: rng.integers(0, 2, n).astype(np.uint16) << 15
+    n = B * L * H
+    big = f32_to_bf16_bits(np.float32(2.0 ** 100))
+    for c in range(128):
+        kind = c % 8
+        col = x[:, :, :, c].reshape(-1).copy()
+        if kind == 1:    # +-2^100 amid unit values: the large terms cancel
+            col[::7] = big
+            col[3::7] = big | np.uint16(0x8000)
+        elif kind == 2:  # any finite bit pattern
+            col = rng.integers(0, 0x7F80, n).astype(np.uint16) | sign(n)
+        elif kind == 3:  # subnormal values only
+            col = rng.integers(1, 0x80, n).astype(np.uint16) | sign(n)
+        elif kind == 4:  # +0 and -0
+            col = np.where(rng.integers(0, 2, n) == 1, 0x8000, 0).astype(np.uint16)
+        elif kind == 5:  # the largest finite values of both signs
+            col = np.uint16(0x7F7F) | sign(n)
+        elif kind == 6:  # any bit pattern, Inf and NaN included (summed as the numbers their bits spell)
+            col = rng.integers(0, 0x10000, n).astype(np.uint16)
+        elif kind == 7:  # unit values with one 2^-39 or 2^-40 value per 64 keys (widest exact span, and one more)
+            col[:] = f32_to_bf16_bits(np.float32(1.0))
+            col[5::64] = f32_to_bf16_bits(np.float32(2.0 ** -39 if c % 16 == 7 else 2.0 ** -40))
+        x[:, :, :, c] = col.reshape(B, L, H)
+    return x
+
+
+@pytest.mark.parametrize("L", [130, 1310])
+def test_recipe_key_mean_is_exact_on_adversarial_channels(L):
+    """The channel means of keys built to defeat a rounded sum (cancellation, subnormals, signed
+    zeros, the largest values, any bit pattern) equal the oracle's exact mean rounded once, bit for
+    bit; 1310 keys also wrap the kernel's 16-stage ring of 64-key slices and end on a ragged one."""
+    B, H = 2, 3
+    k = _adversarial_keys(B, L, H, 20 + L)
+    v = f32_to_bf16_bits(np.random.default_rng(L).standard_normal((B, L, H, 128)).astype(np.float32))
+    cache = KVCache(B, H, L, 2, smooth_k=True)
+    cache.quantize(1, dev_bf16(k), dev_bf16(v))
+    got = cache.k_mean.cpu().numpy()[:, :, 1]
+    want = oracle.key_mean(k)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
 def test_recipe_static_scratch_matches_workspace_call():
     import torch
     w = W["1.3b"]
