@@ -81,6 +81,13 @@ __device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t addr, uint32_
   asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
   return v;
 }
+__device__ __forceinline__ unsigned long long ld_shared_cluster_u64(uint32_t addr, uint32_t rank) {
+  uint32_t remote;
+  unsigned long long v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(rank));
+  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(remote) : "memory");
+  return v;
+}
 
 // ---------------------------------------------------------------- fences
 // Generic-proxy shared-memory writes -> visible to the async proxy (TMA, tensor core).

@@ -238,11 +238,11 @@ __global__ void __launch_bounds__(kThreads, 6) quantize_kernel(const __grid_cons
 // Recipe path, taken by caches with recipe options: K-smoothing of K and adaptive {4, 6}
 // block-scale targets of V (reading note, "The inference infrastructure": both applied within
 // each chunk; "Engineering details of NVFP4 training": candidate scale magnitudes {4, 6}).
-//   key_mean_kernel       one CTA per (32 channels, b, h): TMA brings 64-token slices of the
-//                         chunk's keys into a ring in shared memory; eight warps add them, a lane
-//                         per channel, exactly (an fp64 sum per slice where that is exact, integer
-//                         bins otherwise), and the exact mean rounded once to fp32 is written to
-//                         the slot's k_mean.
+//   key_mean_kernel       a cluster of CTAs per (32 channels, b, h): TMA brings 64-token slices
+//                         of the chunk's keys into a ring in shared memory; eight warps add them, a
+//                         lane per channel, exactly (an fp64 sum per slice where that is exact,
+//                         integer bins otherwise); CTA 0 adds the cluster's bins and writes the
+//                         exact mean rounded once to fp32 to the slot's k_mean.
 //   recipe_amax_kernel    amax_kernel over x - mu for a smoothed K (fp32 magnitudes); the
 //                         partials hold fp32 bit patterns for both tensors.
 //   recipe_encode_kernel  quantize_kernel from x - mu for a smoothed K; for V with adaptive
@@ -332,9 +332,12 @@ __device__ float exact_mean_to_f32(uint32_t (&d)[n], uint32_t L) {
 // once to fp32.  Every bf16 value is a whole number of 2^-133 (< 2^261 of them), so the sum is
 // kept exactly as integers in nine 64-bit bins per channel, bin k counting units of 2^(32 k - 133):
 // integer additions, so any order gives the same sum and the tokens are summed in parallel.
-// One CTA per (32 channels, b, h): a producer lane TMA-loads 64-token x 32-channel boxes into a
-// 16-stage ring; eight warps take the stages in turn, a lane per channel, each thread adding into
-// bins of its own, which are summed at the end.
+// A cluster of S CTAs per (32 channels, b, h), S chosen so the grid fills the SMs: CTA z of the
+// cluster takes the 64-token slices z, z + S, ...; in each CTA a producer lane TMA-loads them
+// (64 tokens x 32 channels) into a 16-stage ring and eight warps take the stages in turn, a lane
+// per channel, each thread adding into bins of its own.  The bins are then summed over the warps,
+// and CTA 0 adds the other CTAs' sums through distributed shared memory (integer additions, so
+// the split changes no bit).
 // A lane first sums its 64 values of a stage in fp64.  When the stage's non-zero magnitudes span
 // at most 40 binades (2^(pos_hi - pos_lo) <= 2^39) every partial sum is a whole number of
 // 2^(pos_lo - 133) below 2^(8 + 39 + 6) = 2^53, so fp64 holds each one exactly, in any order; the
@@ -361,10 +364,13 @@ __global__ void __launch_bounds__(32 * (kMeanWarps + 1)) key_mean_kernel(const _
   __shared__ unsigned long long bins[kMeanWarps][kMeanBins][kMeanCh];  // each slot owned by one thread
   __shared__ int s_issued;
   __shared__ int s_bad;
+  __shared__ int s_ok;  // this CTA summed all of its slices
   const int cg = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = (a.L + kMeanTok - 1) / kMeanTok;
+  const int split = blockIdx.z, n_split = gridDim.z;  // cluster (1, 1, n_split): rank = split
+  const int all_tiles = (a.L + kMeanTok - 1) / kMeanTok;
+  const int n_tiles = split < all_tiles ? (all_tiles - split + n_split - 1) / n_split : 0;  // this CTA's
   for (int i = threadIdx.x; i < kMeanWarps * kMeanBins * kMeanCh; i += blockDim.x) (&bins[0][0][0])[i] = 0ull;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMeanStages; ++i) {
@@ -389,8 +395,8 @@ __global__ void __launch_bounds__(32 * (kMeanWarps + 1)) key_mean_kernel(const _
           break;
         }
         ptx::mbar_arrive_expect_tx(ptx::smem_u32(&full[st]), kMeanTok * kMeanCh * 2);
-        ptx::tma_load_4d(ptx::smem_u32(ring + st * kMeanTok * kMeanCh), &tm, cg * kMeanCh, h, i * kMeanTok, b,
-                         ptx::smem_u32(&full[st]));
+        ptx::tma_load_4d(ptx::smem_u32(ring + st * kMeanTok * kMeanCh), &tm, cg * kMeanCh, h,
+                         (split + i * n_split) * kMeanTok, b, ptx::smem_u32(&full[st]));
         ++issued;
       }
       s_issued = issued;
@@ -402,7 +408,7 @@ __global__ void __launch_bounds__(32 * (kMeanWarps + 1)) key_mean_kernel(const _
       const int st = i % kMeanStages;
       ok = __all_sync(0xFFFFFFFFu, wait_phase(ptx::smem_u32(&full[st]), (i / kMeanStages) & 1));
       if (!ok) break;
-      const int n = min(kMeanTok, a.L - i * kMeanTok);
+      const int n = min(kMeanTok, a.L - (split + i * n_split) * kMeanTok);
       const uint16_t* col = ring + st * kMeanTok * kMeanCh + lane;
       // fp64 sum of the stage, with the largest magnitude and the smallest non-zero one (as bit
       // patterns: a zero's pattern less one wraps to the top and never wins the minimum)
@@ -478,29 +484,56 @@ __global__ void __launch_bounds__(32 * (kMeanWarps + 1)) key_mean_kernel(const _
   }
   if (!ok && lane == 0) atomicOr(a.status, kStatusTimeout);
   __syncthreads();
-  if (warp == 0 && s_bad == 0 && s_issued == n_tiles) {
-    // S = sum over bins of bins[k] * 2^(32 k) as 32-bit digits (two's complement), then the mean
-    constexpr int kDigits = kMeanBins + 1;
-    uint32_t d[kDigits];
-    int64_t carry = 0;
-#pragma unroll
-    for (int k = 0; k < kDigits; ++k) {
-      unsigned long long bk = 0ull;  // bin k of this channel over the warps (wrapping sum)
-      if (k < kMeanBins)
-#pragma unroll
-        for (int w = 0; w < kMeanWarps; ++w) bk += bins[w][k][lane];
-      const int64_t acc = carry + static_cast<int64_t>(bk);
-      d[k] = static_cast<uint32_t>(acc);           // the low 32 bits
-      carry = (acc - static_cast<int64_t>(d[k])) / (int64_t(1) << 32);  // exact: the rest is a multiple
-    }
-    a.k_mean[(static_cast<int64_t>(bh) * a.C + a.slot) * kHeadDim + cg * kMeanCh + lane] =
-        exact_mean_to_f32<kDigits>(d, static_cast<uint32_t>(a.L));
-  }
   if (threadIdx.x == 32 * kMeanWarps) {
     // after a time-out some copies may still be in flight: let them land (bounded) before the
     // CTA's shared memory goes away
     for (int i = max(0, s_issued - kMeanStages); i < s_issued; ++i)
       if (!wait_phase(ptx::smem_u32(&full[i % kMeanStages]), (i / kMeanStages) & 1)) break;
+  }
+  if (warp == 0) {
+    // this CTA's sum per bin: the warps' bins added into warp 0's (wrapping sums)
+#pragma unroll
+    for (int k = 0; k < kMeanBins; ++k) {
+      unsigned long long bk = bins[0][k][lane];
+#pragma unroll
+      for (int w = 1; w < kMeanWarps; ++w) bk += bins[w][k][lane];
+      bins[0][k][lane] = bk;
+    }
+    if (lane == 0) s_ok = (s_bad == 0 && s_issued == n_tiles) ? 1 : 0;
+  }
+  __syncthreads();
+  if (n_split > 1) {  // every CTA's sums visible to the cluster
+    ptx::cluster_arrive_release();
+    ptx::cluster_wait_acquire();
+  }
+  if (split == 0 && warp == 0) {
+    unsigned long long bk[kMeanBins];
+#pragma unroll
+    for (int k = 0; k < kMeanBins; ++k) bk[k] = bins[0][k][lane];
+    bool all_ok = s_ok != 0;
+    for (int r = 1; r < n_split; ++r) {
+      all_ok = all_ok && ptx::ld_shared_cluster_u32(ptx::smem_u32(&s_ok), r) != 0u;
+#pragma unroll
+      for (int k = 0; k < kMeanBins; ++k) bk[k] += ptx::ld_shared_cluster_u64(ptx::smem_u32(&bins[0][k][lane]), r);
+    }
+    if (all_ok) {
+      // S = sum over bins of bk[k] * 2^(32 k) as 32-bit digits (two's complement), then the mean
+      constexpr int kDigits = kMeanBins + 1;
+      uint32_t d[kDigits];
+      int64_t carry = 0;
+#pragma unroll
+      for (int k = 0; k < kDigits; ++k) {
+        const int64_t acc = carry + (k < kMeanBins ? static_cast<int64_t>(bk[k]) : 0);
+        d[k] = static_cast<uint32_t>(acc);                                // the low 32 bits
+        carry = (acc - static_cast<int64_t>(d[k])) / (int64_t(1) << 32);  // exact: the rest is a multiple
+      }
+      a.k_mean[(static_cast<int64_t>(bh) * a.C + a.slot) * kHeadDim + cg * kMeanCh + lane] =
+          exact_mean_to_f32<kDigits>(d, static_cast<uint32_t>(a.L));
+    }
+  }
+  if (n_split > 1) {  // CTA 0 has read the others' shared memory
+    ptx::cluster_arrive_release();
+    ptx::cluster_wait_acquire();
   }
 }
 
@@ -1160,6 +1193,18 @@ cudaError_t launch_encode_dependent(Kernel kernel, const QuantArgs& a, cudaStrea
 
 PerDeviceOnce g_mean_attr;
 
+// CTAs per (32 channels, b, h) of the channel-mean grid: enough to fill the SMs once, at most 8 (a
+// portable cluster), and at least four 64-token slices each.
+unsigned mean_splits(const nvfp4kv_cache& c) {
+  const int sms = current_sm_count();
+  const int64_t ctas = static_cast<int64_t>(kHeadDim / kMeanCh) * c.batch * c.heads;
+  const int64_t slices = (c.chunk_tokens + kMeanTok - 1) / kMeanTok;
+  int64_t s = sms > 0 ? sms / ctas : 1;
+  s = std::min<int64_t>(s, 8);
+  s = std::min<int64_t>(s, slices / 4);
+  return static_cast<unsigned>(std::max<int64_t>(s, 1));
+}
+
 cudaError_t launch_quantize_recipe(const nvfp4kv_cache& c, int slot, const uint16_t* k, const uint16_t* v,
                                    int64_t token_stride, void* workspace, cudaStream_t stream) {
   const QuantArgs a = two_pass_args(c, slot, k, v, token_stride, workspace);
@@ -1189,8 +1234,19 @@ cudaError_t launch_quantize_recipe(const nvfp4kv_cache& c, int slot, const uint1
                                   static_cast<int>(kMeanSmem));
     });
     if (attr_err != cudaSuccess) return attr_err;
-    key_mean_kernel<<<dim3(kHeadDim / kMeanCh, c.batch * c.heads), 32 * (kMeanWarps + 1), kMeanSmem, stream>>>(tm, m);
-    const cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kHeadDim / kMeanCh, c.batch * c.heads, mean_splits(c));
+    cfg.blockDim = dim3(32 * (kMeanWarps + 1), 1, 1);
+    cfg.dynamicSmemBytes = kMeanSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = cfg.gridDim.z;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, key_mean_kernel, tm, m);
     if (e != cudaSuccess) return e;
   }
   recipe_amax_kernel<<<dim3(a.parts, c.batch * c.heads, 2), kThreads, 0, stream>>>(a);

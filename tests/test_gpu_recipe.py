@@ -127,12 +127,12 @@ def _adversarial_keys(B, L, H, seed):
     return x
 
 
-@pytest.mark.parametrize("L", [130, 1310])
-def test_recipe_key_mean_is_exact_on_adversarial_channels(L):
+@pytest.mark.parametrize("B,H,L", [(2, 3, 130), (2, 3, 1310), (1, 1, 10000)])
+def test_recipe_key_mean_is_exact_on_adversarial_channels(B, H, L):
     """The channel means of keys built to defeat a rounded sum (cancellation, subnormals, signed
     zeros, the largest values, any bit pattern) equal the oracle's exact mean rounded once, bit for
-    bit; 1310 keys also wrap the kernel's 16-stage ring of 64-key slices and end on a ragged one."""
-    B, H = 2, 3
+    bit.  1310 and 10000 keys end on a ragged 64-key slice and are split over a cluster of CTAs on a
+    GPU with enough SMs; 10000 keys on one head also wrap each CTA's 16-stage ring."""
     k = _adversarial_keys(B, L, H, 20 + L)
     v = f32_to_bf16_bits(np.random.default_rng(L).standard_normal((B, L, H, 128)).astype(np.float32))
     cache = KVCache(B, H, L, 2, smooth_k=True)
